@@ -1,0 +1,121 @@
+"""fp64 CPU oracle for tree-verification attention — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The CUDA product path never does, and the
+two share no code; they meet only at the seeded inputs.
+
+``verify_attn_oracle`` is one softmax over prefix U ancestors-or-self per query
+row (LongSpec, gist.science summary, section 2C), computed in fp64 from the exact
+bf16 inputs by ``verify_attn_oracle.c``. ``softmax_keyset`` is the same softmax over
+an explicit key list, used by the tests to check the log-sum-exp merge.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        lib.oracle_verify_attn.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_double, P, ctypes.c_int64, P, P,
+                                           ctypes.c_int]
+        lib.oracle_verify_attn.restype = ctypes.c_int
+        lib.oracle_softmax_keyset.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_int, ctypes.c_double, P, P]
+        lib.oracle_softmax_keyset.restype = None
+        lib.oracle_check_trees.argtypes = [P, ctypes.c_int, ctypes.c_int]
+        lib.oracle_check_trees.restype = ctypes.c_int
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def verify_attn_oracle(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens,
+                       *, num_q_heads: int, num_kv_heads: int, head_dim: int, tree_size: int,
+                       scale: Optional[float] = None, rows: Optional[np.ndarray] = None,
+                       nthreads: int = 0):
+    """Returns (out fp64 [n, d], lse fp64 [n]) for the selected rows.
+
+    Row r = (b*T + i)*H_q + h. rows=None computes all B*T*H_q rows in that order.
+    Tensors are bf16 bit patterns (uint16) in the C-ABI layouts.
+    """
+    lib = _load()
+    d, T = head_dim, tree_size
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    B = len(cu) - 1
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (q, k_cache, v_cache, k_tree, v_tree)]
+    par = np.ascontiguousarray(parent, dtype=np.int32)
+    if rows is None:
+        n = B * T * num_q_heads
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n = len(rows_arr)
+    out = np.empty((n, d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    rc = lib.oracle_verify_attn(*[_ptr(a) for a in arrs], _ptr(par), _ptr(cu), B, num_q_heads,
+                                num_kv_heads, d, T, float(scale),
+                                None if rows_arr is None else _ptr(rows_arr), n,
+                                _ptr(out), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise OracleError({1: "bad argument", 2: "bad tree", 3: "out of memory"}.get(rc, rc))
+    return out, lse
+
+
+def verify_attn_oracle_inputs(inp, rows=None, nthreads: int = 0, scale=None):
+    """Convenience: run the oracle on an ``inputs.Inputs`` bundle."""
+    w = inp.workload
+    return verify_attn_oracle(inp.q, inp.k_cache, inp.v_cache, inp.k_tree, inp.v_tree,
+                              inp.parent, inp.cu_seqlens, num_q_heads=w.num_q_heads,
+                              num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                              tree_size=w.tree_size, scale=scale if scale is not None else inp.scale,
+                              rows=rows, nthreads=nthreads)
+
+
+def softmax_keyset(q_row, keys, vals, scale: float):
+    """One fp64 softmax of a bf16 query row over bf16 key/value rows [n, d]."""
+    lib = _load()
+    q_row = np.ascontiguousarray(q_row, dtype=np.uint16)
+    keys = np.ascontiguousarray(keys, dtype=np.uint16).reshape(-1, q_row.shape[-1])
+    vals = np.ascontiguousarray(vals, dtype=np.uint16).reshape(-1, q_row.shape[-1])
+    d = q_row.shape[-1]
+    out = np.empty(d, dtype=np.float64)
+    lse = np.empty(1, dtype=np.float64)
+    lib.oracle_softmax_keyset(_ptr(q_row), _ptr(keys), _ptr(vals), keys.shape[0], d, d,
+                              float(scale), _ptr(out), _ptr(lse))
+    return out, float(lse[0])
+
+
+def check_trees(parent, B: int, T: int) -> bool:
+    par = np.ascontiguousarray(parent, dtype=np.int32)
+    return _load().oracle_check_trees(_ptr(par), B, T) == 0
+
+
+__all__ = ["verify_attn_oracle", "verify_attn_oracle_inputs", "softmax_keyset", "check_trees",
+           "max_threads", "OracleError"]
