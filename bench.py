@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of tree-verification attention (LongSpec hybrid tree attention) on B200.
+
+One step = one full verification-attention call (prefix partials + tree/combine) over one
+batch of synthetic input of the named workload, inputs resident in HBM. L2 is flushed
+(a write of twice the L2 size) before every timed step, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+N > 1 runs under torchrun: every rank runs an independent problem of the same workload
+on its own GPU (replicas, weak scaling, no collective on the data path); the step time
+is the max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from tree_verification_attention_longspec_b200.inputs import make_inputs  # noqa: E402
+from tree_verification_attention_longspec_b200.workloads import (  # noqa: E402
+    HEADLINE, WORKLOADS, algorithmic_bytes, algorithmic_flops)
+
+METRIC = "verify-attn µs/call and KV HBM GB/s (% roofline) at L=64k, T=64, bf16"
+UNIT = "us/call"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DOMINANT_KERNEL_SRC = os.path.join(ROOT, "tree_verification_attention_longspec_b200", "csrc")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_figures(inp):
+    w = inp.workload
+    L = inp.prefix_lengths
+    total_L = int(L.sum())
+    step_bytes = algorithmic_bytes(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.tree_size,
+                                   total_L)
+    step_flops = algorithmic_flops(w.num_q_heads, w.head_dim, w.tree_size, L)
+    # the prefix kernel alone: every (query row, prefix key) pair costs 4*d flops, and the
+    # prefix K/V plus the queries are its compulsory bytes
+    rows = w.batch * w.tree_size * w.num_q_heads
+    prefix_flops = 4 * w.head_dim * w.tree_size * w.num_q_heads * total_L
+    prefix_bytes = 4 * total_L * w.num_kv_heads * w.head_dim + 2 * rows * w.head_dim
+    kv_bytes = 4 * total_L * w.num_kv_heads * w.head_dim
+    return dict(total_L=total_L, step_bytes=step_bytes, step_flops=step_flops,
+                prefix_flops=prefix_flops, prefix_bytes=prefix_bytes, kv_bytes=kv_bytes, rows=rows)
+
+
+def config_of(inp, l2_note):
+    w = inp.workload
+    L = inp.prefix_lengths
+    return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "tree_size": w.tree_size,
+            "tree": w.tree, "prefix_len": int(L[0]) if len(set(L.tolist())) == 1 else "ragged",
+            "total_prefix_len": int(L.sum()), "seed": inp.seed, "l2": l2_note}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU through NVML in a thread."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report without clocks
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((mhz, rs, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        reasons = set()
+        for _, rs, _ in loaded:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        med = statistics.median([s[0] for s in loaded]) if loaded else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "samples_under_load": len([s for s in self.samples if s[2] > 0])}
+
+
+# ----------------------------------------------------------------------------- traffic record
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(DOMINANT_KERNEL_SRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(DOMINANT_KERNEL_SRC, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch of the prefix kernel from the committed ncu summary, when it
+    was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        r = rec.get(workload_name)
+        if r and r.get("source_hash") == kernel_source_hash():
+            return r.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def time_oracle(inp, target_s=12.0, max_rows=None):
+    """Time the fp64 oracle on a bounded sample of rows with every host core; returns
+    (us per full call, rows sampled, seconds, cores)."""
+    import oracle
+    w = inp.workload
+    total = w.batch * w.tree_size * w.num_q_heads
+    cores = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(123)
+    probe = np.sort(rng.choice(total, size=min(total, max(cores, 8)), replace=False))
+    t0 = time.perf_counter()
+    oracle.verify_attn_oracle_inputs(inp, rows=probe, nthreads=cores)
+    t_probe = max(time.perf_counter() - t0, 1e-6)
+    per_row = t_probe / len(probe)
+    n = int(min(total, max(len(probe), target_s / per_row)))
+    if max_rows:
+        n = min(n, max_rows)
+    rows = np.sort(rng.choice(total, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.verify_attn_oracle_inputs(inp, rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    return dt / n * total * 1e6, n, dt, cores
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, seed=0)
+    total = w.batch * w.tree_size * w.num_q_heads
+    per_step_target = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    n_rows = cores = None
+    for s in range(args.warmup + args.steps):
+        us, n_rows, dt, cores = time_oracle(inp, target_s=per_step_target)
+        if s >= args.warmup:
+            vals.append(us)
+    v = float(statistics.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(inp, "n/a (CPU)"),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{n_rows} of {total} query rows per step, scaled to one call"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from tree_verification_attention_longspec_b200 import binding
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load_library()
+
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, seed=rank)   # independent problem per rank
+    fig = workload_figures(inp)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+
+    d_in = dict(q=bf(inp.q), k_cache=bf(inp.k_cache), v_cache=bf(inp.v_cache), k_tree=bf(inp.k_tree),
+                v_tree=bf(inp.v_tree), parent=i32(inp.parent), cu=i32(inp.cu_seqlens))
+    op = binding.VerifyAttn(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.tree_size,
+                            cu_seqlens_host=inp.cu_seqlens, device=dev)
+    out = torch.empty_like(d_in["q"])
+    lse = torch.empty(out.shape[0], w.num_q_heads, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    ptr = {k: v.data_ptr() for k, v in d_in.items()}
+    dims, ws, wsb = op.dims, op.workspace.data_ptr(), op.ws_bytes
+
+    def prefix():
+        rc = binding.call_prefix_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["cu"], dims, ws,
+                                     wsb, sp)
+        if rc:
+            raise binding.LSError(rc, "ls_verify_attn_prefix")
+
+    def tree_combine():
+        rc = binding.call_tree_combine_raw(ptr["q"], ptr["k_tree"], ptr["v_tree"], ptr["parent"],
+                                           ptr["cu"], out.data_ptr(), lse.data_ptr(), dims, ws, wsb, sp)
+        if rc:
+            raise binding.LSError(rc, "ls_verify_attn_tree_combine")
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        prefix()
+        tree_combine()
+    torch.cuda.synchronize(dev)
+    st = op.check()
+    if st != 0:
+        raise binding.LSError(st, "device status after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        for k in range(K):
+            flush.zero_()
+            ev[k][0].record(stream)
+            prefix()
+            ev[k][1].record(stream)
+            tree_combine()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    prefix_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    ms_per_step = float(statistics.mean(step_ms))
+    prefix_avg_ms = float(statistics.mean(prefix_ms))
+    if world > 1:
+        t = torch.tensor([ms_per_step, prefix_avg_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step, prefix_avg_ms = float(t[0]), float(t[1])
+    st = op.check()
+    if st != 0:
+        raise binding.LSError(st, "device status after timing")
+
+    # e2e through the public call with host buffers: H2D of every input, the call, D2H of out+lse
+    e2e = None
+    if not args.no_e2e:
+        h_in = {k: v.cpu().pin_memory() for k, v in d_in.items()}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        d2 = {k: torch.empty_like(v) for k, v in d_in.items()}
+        h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+        d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+        n_e2e = max(3, min(K, 20))
+        times = []
+        for k in range(2 + n_e2e):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            e0.record(stream)
+            for name in d2:
+                d2[name].copy_(h_in[name], non_blocking=True)
+            o2, l2_ = op(d2["q"], d2["k_cache"], d2["v_cache"], d2["k_tree"], d2["v_tree"], d2["parent"],
+                         d2["cu"], out, lse)
+            h_out.copy_(o2, non_blocking=True)
+            h_lse.copy_(l2_, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if k >= 2:
+                times.append(e0.elapsed_time(e1))
+        e2e_ms = float(statistics.mean(times))
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        e2e = {"value": e2e_ms * 1000.0 / world, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    prefix_s = prefix_avg_ms / 1000.0
+    t_bytes = fig["prefix_bytes"] / (hbm * 1e9)
+    t_flops = fig["prefix_flops"] / (tc * 1e12)
+    if t_flops >= t_bytes:
+        roof = {"bound": "tensor", "achieved": fig["prefix_flops"] / prefix_s / 1e12, "peak": tc,
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": fig["prefix_bytes"] / prefix_s / 1e9, "peak": hbm,
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(w.name)
+    roof["kernel"] = "prefix (ls_verify_attn_prefix)"
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured" else "fallback"
+    roof["kernel_us"] = prefix_avg_ms * 1000.0
+    step_s = ms_per_step / 1000.0
+    roof_step_s = max(fig["step_bytes"] / (hbm * 1e9), fig["step_flops"] / (tc * 1e12))
+
+    line = {"metric": METRIC, "value": ms_per_step * 1000.0 / world, "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16, random draft trees)",
+            "config": config_of(inp, "flushed before every step (write of 2x L2), outside the timed events"),
+            "kv_hbm_gbs": fig["kv_bytes"] / step_s / 1e9,
+            "roofline_step": {"roofline_us": roof_step_s * 1e6, "frac": roof_step_s / step_s,
+                              "bytes": fig["step_bytes"], "flops": fig["step_flops"]},
+            "roofline": roof, "gpu_launches": 2 * K, "plan": op.plan,
+            "clocks": sampler.summary(), "e2e": e2e}
+    if world == 1 and not args.no_cpu_baseline:
+        us, n, dt, cores = time_oracle(inp, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{n} of {fig['rows']} query rows ({dt:.1f} s), scaled to one call"}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE.name, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

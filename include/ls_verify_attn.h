@@ -1,0 +1,161 @@
+/*
+ * ls_verify_attn — tree-verification attention for long-context speculative decoding,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation (LongSpec: Long-Context Lossless Speculative Decoding with Efficient
+ * Drafting and Verification; gist.science summary, section 2C "Schnelle Tree
+ * Attention", the "Aufteilung" and "Aggregation" paragraphs): every query token of a
+ * speculated token tree attends
+ *   - to the whole cached prefix of its sequence, with no mask ("Cached-Teil"), and
+ *   - to the tree tokens under the tree mask ("Speculative-Teil"), read here as
+ *     ancestor-or-self visibility built from a parent[] array,
+ * and the two partial softmax results are merged with a log-sum-exp step so that
+ * the output equals one softmax over the union of both key sets. The abstracts
+ * (arXiv v1 on mlsanity; ACL record on PaperTrail) call the method lossless: the
+ * result is exact attention, not an approximation.
+ *
+ * For sequence b, tree node i, query head h (kv head kh = h / (H_q / H_kv)):
+ *   visible(i) = { prefix keys 0..L_b-1 } U { tree nodes a : a == i or a is an ancestor of i }
+ *   s_x  = softmax_scale * <q[b,i,h,:], k_x[kh,:]>
+ *   lse  = ln sum_{x in visible(i)} exp(s_x)            (natural log, scale included)
+ *   out  = sum_{x in visible(i)} exp(s_x - lse) * v_x[kh,:]
+ *
+ * All calls are C functions with plain pointers and sizes. Device pointers are CUDA
+ * device (or managed) memory of the current device. The library allocates no memory
+ * and keeps no state between calls; every buffer, including the workspace, belongs
+ * to the caller. Nothing in this library traps or aborts: errors come back as status
+ * codes.
+ */
+#ifndef LS_VERIFY_ATTN_H
+#define LS_VERIFY_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LS_API __attribute__((visibility("default")))
+#else
+#define LS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+enum {
+  LS_OK = 0,
+  LS_ERR_INVALID_ARG = 1,  /* null pointer, bad dimension, misaligned pointer, bad cu_seqlens_host */
+  LS_ERR_UNSUPPORTED = 2,  /* head_dim other than 64/128, tree_size > 128, not an sm_100 device */
+  LS_ERR_WORKSPACE = 3,    /* workspace null, misaligned or smaller than ls_verify_attn_workspace_size */
+  LS_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
+  LS_ERR_BAD_TREE = 5,     /* device found parent[] that is not a rooted tree with parent[i] < i */
+  LS_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up (pipeline stalled) */
+  LS_ERR_LENGTHS = 7       /* device cu_seqlens disagrees with cu_seqlens_host / max_prefix_len */
+};
+
+/* Problem description, passed by pointer to every call. */
+typedef struct ls_verify_dims {
+  int32_t batch;          /* B >= 1 sequences */
+  int32_t num_q_heads;    /* H_q >= 1, a multiple of num_kv_heads (grouped-query attention) */
+  int32_t num_kv_heads;   /* H_kv >= 1 */
+  int32_t head_dim;       /* d: 64 or 128 */
+  int32_t tree_size;      /* T: tree nodes per sequence, 1..128, the same for every sequence */
+  int32_t max_prefix_len; /* an upper bound on every L_b (used when cu_seqlens_host is NULL) */
+  const int32_t* cu_seqlens_host; /* optional HOST copy of cu_seqlens [B+1]; when given it must
+                                     equal the device array, and the work split is balanced
+                                     over the actual lengths. NULL: every sequence is planned
+                                     as max_prefix_len long (correct, less balanced). */
+  float softmax_scale;    /* <= 0 selects 1/sqrt(head_dim) */
+} ls_verify_dims;
+
+/*
+ * Bytes of device workspace that ls_verify_attn needs for these dims on the current
+ * device (it depends on the SM count and, when cu_seqlens_host is given, on the
+ * lengths). Returns 0 if the dims are invalid or unsupported.
+ */
+LS_API size_t ls_verify_attn_workspace_size(const ls_verify_dims* dims);
+
+/*
+ * Tree-verification attention, asynchronous on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream). Returns after enqueuing its kernels.
+ *
+ *   q          bf16 [B*T, H_q, d]      tree queries, token-major (row b*T+i is node i
+ *                                      of sequence b), already position-encoded
+ *   k_cache    bf16 [sum_b L_b, H_kv, d] prefix keys of all sequences, packed in
+ *                                      sequence order by cu_seqlens
+ *   v_cache    bf16 [sum_b L_b, H_kv, d]
+ *   k_tree     bf16 [B*T, H_kv, d]     keys of the tree tokens
+ *   v_tree     bf16 [B*T, H_kv, d]
+ *   tree_parent int32 [B*T]            parent of node i of sequence b as a local index:
+ *                                      -1 for node 0 (the root), in [0, i) otherwise
+ *   cu_seqlens int32 [B+1] (device)    cu_seqlens[0] = 0, L_b = cu[b+1] - cu[b] >= 0
+ *   out        bf16 [B*T, H_q, d]      written (round to nearest even)
+ *   lse        fp32 [B*T, H_q]         written: natural-log normaliser, scale included
+ *   workspace  device scratch of at least ls_verify_attn_workspace_size(dims) bytes,
+ *              256-byte aligned; its contents need no initialisation and are
+ *              overwritten. Concurrent calls must use different workspaces.
+ *
+ * Every tensor is dense row-major with the innermost dimension contiguous. The bf16
+ * tensors must start on a 16-byte boundary, the int32/fp32 ones on a 4-byte boundary. `out` and `lse` must not alias any input.
+ * Host-detectable errors return LS_ERR_INVALID_ARG / LS_ERR_UNSUPPORTED /
+ * LS_ERR_WORKSPACE before anything is launched. Errors that only the device can see
+ * (bad tree, cu_seqlens mismatch, a wait that timed out) are recorded in the
+ * workspace and reported by ls_verify_attn_check; the outputs of such a call are
+ * unspecified but no memory outside the given buffers is touched.
+ */
+LS_API int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache,
+                   const void* k_tree, const void* v_tree,
+                   const int32_t* tree_parent, const int32_t* cu_seqlens,
+                   void* out, float* lse,
+                   const ls_verify_dims* dims,
+                   void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/*
+ * The two stages that ls_verify_attn runs, for callers that want to place or time
+ * them separately. They must be called in this order, on the same stream (or with
+ * the caller ordering them), with the same dims and workspace; together they are
+ * exactly ls_verify_attn. Arguments as for ls_verify_attn.
+ *
+ * ls_verify_attn_prefix (the "Cached-Teil" of section 2C): attention of every tree
+ * query over its sequence's cached prefix with no mask. The prefix is split into
+ * chunks of 128-key blocks; each chunk leaves a partial (out normalised by its own
+ * sum, lse) in the workspace.
+ *
+ * ls_verify_attn_tree_combine (the "Speculative-Teil" and "Aggregation" of section
+ * 2C): builds each node's ancestor-or-self set from tree_parent, attends over those
+ * tree keys, merges the result with every prefix partial by log-sum-exp, and writes
+ * `out` and `lse`.
+ */
+LS_API int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* cu_seqlens, const ls_verify_dims* dims,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+LS_API int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const void* v_tree,
+                                       const int32_t* tree_parent, const int32_t* cu_seqlens,
+                                       void* out, float* lse, const ls_verify_dims* dims,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Waits for `stream`, then reads the device-side status that the last ls_verify_attn
+ * call with this workspace and these dims recorded. Returns LS_OK, LS_ERR_BAD_TREE,
+ * LS_ERR_LENGTHS, LS_ERR_TIMEOUT, or LS_ERR_CUDA if the copy itself failed.
+ */
+LS_API int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void* stream);
+
+/* A static, human-readable name for a status code. */
+LS_API const char* ls_status_string(int status);
+
+/*
+ * Describes how ls_verify_attn splits the work for these dims on the current device:
+ * number of prefix work units (CTAs of the prefix kernel), 128-key blocks per unit,
+ * and CTAs of the tree/combine kernel. Any pointer may be NULL. Returns a status.
+ */
+LS_API int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* prefix_ctas,
+                        int32_t* blocks_per_chunk, int32_t* combine_ctas);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LS_VERIFY_ATTN_H */

@@ -22,6 +22,7 @@ def gpu_available() -> bool:
 
 @pytest.fixture(scope="session")
 def cuda_lib():
-    """The C-ABI library, loaded through the binding (raises if it is not built)."""
-    from tree_verification_attention_longspec_b200 import binding
+    """The C-ABI library, built in-tree if needed and loaded through the binding."""
+    from tree_verification_attention_longspec_b200 import binding, build
+    build.build()
     return binding.load_library()

@@ -1,0 +1,69 @@
+"""Shared helpers for the GPU tests: move a seeded input bundle to the device, run the
+C-ABI path, and pick sample rows for the oracle."""
+from __future__ import annotations
+
+import numpy as np
+
+OUT_ATOL = 1e-2   # max-abs error on bf16 `out` against the fp64 oracle
+LSE_ATOL = 1e-3   # max-abs error on fp32 `lse`
+
+
+def to_device(inp, device="cuda:0"):
+    import torch
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+    return dict(q=bf(inp.q), k_cache=bf(inp.k_cache), v_cache=bf(inp.v_cache), k_tree=bf(inp.k_tree),
+                v_tree=bf(inp.v_tree), parent=i32(inp.parent), cu_seqlens=i32(inp.cu_seqlens))
+
+
+def make_op(inp, host_lengths=True, scale=0.0, max_prefix_len=None):
+    from tree_verification_attention_longspec_b200.binding import VerifyAttn
+    w = inp.workload
+    L = np.diff(inp.cu_seqlens)
+    mpl = int(L.max()) if max_prefix_len is None else max_prefix_len
+    return VerifyAttn(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.tree_size,
+                      cu_seqlens_host=inp.cu_seqlens if host_lengths else None, max_prefix_len=mpl,
+                      softmax_scale=scale)
+
+
+def run_gpu(inp, host_lengths=True, scale=0.0, dev=None, op=None):
+    """Returns (out fp64 [B*T*H_q, d], lse fp64 [B*T*H_q], device status)."""
+    import torch
+    if dev is None:
+        dev = to_device(inp)
+    if op is None:
+        op = make_op(inp, host_lengths, scale)
+    out, lse = op(dev["q"], dev["k_cache"], dev["v_cache"], dev["k_tree"], dev["v_tree"],
+                  dev["parent"], dev["cu_seqlens"])
+    torch.cuda.synchronize()
+    status = op.check()
+    w = inp.workload
+    o = out.float().cpu().numpy().astype(np.float64).reshape(-1, w.head_dim)
+    l = lse.cpu().numpy().astype(np.float64).reshape(-1)
+    return o, l, status
+
+
+def sample_rows(inp, n_random=48, seed=0):
+    """Rows r = (b*T+i)*H_q + h covering the first/last node and head of every sequence,
+    the first and last row of every 256-row group of every kv head, plus random rows."""
+    w = inp.workload
+    B, T, Hq, Hkv = w.batch, w.tree_size, w.num_q_heads, w.num_kv_heads
+    g = Hq // Hkv
+    rows = set()
+    for b in range(B):
+        for i in (0, T - 1):
+            for h in (0, Hq - 1):
+                rows.add((b * T + i) * Hq + h)
+        for kh in range(Hkv):
+            for r_local in range(0, T * g, 256):
+                for rr in (r_local, min(r_local + 255, T * g - 1)):
+                    i, j = divmod(rr, g)
+                    rows.add((b * T + i) * Hq + kh * g + j)
+    rng = np.random.default_rng(seed)
+    rows.update(int(x) for x in rng.integers(0, B * T * Hq, size=n_random))
+    return np.array(sorted(rows), dtype=np.int64)

@@ -1,0 +1,62 @@
+// Host-side check of the chunk plan: every (sequence, kv head, row group, 128-key
+// block) of the prefix is covered by exactly one chunk, chunk ids are dense, and the
+// per-sequence chunk ranges that the combine kernel uses agree with locate_chunk.
+// Usage: plan_check B Hq Hkv T C uniform_n L_0 ... L_{B-1}   (exit 0 = pass)
+#include <cstdio>
+#include <cstdlib>
+#include <map>
+#include <tuple>
+#include <vector>
+
+#include "ls_plan.cuh"
+
+int main(int argc, char** argv) {
+  if (argc < 7) return 2;
+  ls::Plan p{};
+  p.B = atoi(argv[1]);
+  p.Hq = atoi(argv[2]);
+  p.Hkv = atoi(argv[3]);
+  p.T = atoi(argv[4]);
+  p.C = atoi(argv[5]);
+  p.uniform_n = atoi(argv[6]);
+  p.d = 128;
+  p.g = p.Hq / p.Hkv;
+  p.rows = p.T * p.g;
+  p.rg = ls::ceil_div(p.rows, ls::kUnitRows);
+  if (argc != 7 + p.B) return 2;
+  std::vector<int32_t> cu(p.B + 1, 0);
+  for (int b = 0; b < p.B; ++b) cu[b + 1] = cu[b] + atoi(argv[7 + b]);
+  int32_t total = 0, first = 0, per = 0;
+  ls::sequence_chunks(p, cu.data(), 0, &first, &per, &total);
+  p.n_chunks = total;
+  std::map<std::tuple<int, int, int, int>, int> seen;  // (b, kh, rg, block) -> count
+  for (int cid = 0; cid < total; ++cid) {
+    ls::ChunkCoord c = ls::locate_chunk(p, cu.data(), cid);
+    if (!c.valid) { printf("chunk %d invalid\n", cid); return 1; }
+    int32_t f, n, t;
+    ls::sequence_chunks(p, cu.data(), c.b, &f, &n, &t);
+    const int expect = f + (c.kh * p.rg + c.rgi) * n + c.split;
+    if (expect != cid) { printf("chunk %d: combine index %d\n", cid, expect); return 1; }
+    if (c.key_end > c.key_begin && c.key_begin % ls::kBlockN) { printf("chunk %d unaligned start\n", cid); return 1; }
+    if (c.key_end - c.key_begin > p.C * ls::kBlockN) { printf("chunk %d too long\n", cid); return 1; }
+    if (c.seq_offset != cu[c.b]) return 1;
+    for (int k = c.key_begin; k < c.key_end; k += ls::kBlockN)
+      seen[std::make_tuple(c.b, c.kh, c.rgi, k / ls::kBlockN)]++;
+  }
+  if (ls::locate_chunk(p, cu.data(), total).valid) { printf("chunk past the end is valid\n"); return 1; }
+  for (int b = 0; b < p.B; ++b) {
+    const int L = cu[b + 1] - cu[b];
+    for (int kh = 0; kh < p.Hkv; ++kh)
+      for (int r = 0; r < p.rg; ++r)
+        for (int k = 0; k < ls::ceil_div(L, ls::kBlockN); ++k) {
+          auto it = seen.find(std::make_tuple(b, kh, r, k));
+          if (it == seen.end() || it->second != 1) {
+            printf("block (%d,%d,%d,%d) covered %d times\n", b, kh, r, k,
+                   it == seen.end() ? 0 : it->second);
+            return 1;
+          }
+        }
+  }
+  printf("ok %d chunks\n", total);
+  return 0;
+}

@@ -1,0 +1,270 @@
+// C-ABI entry points: argument checks, the work split, workspace layout and launches.
+// Declared and documented in include/ls_verify_attn.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <vector>
+
+#include "ls_device.cuh"
+#include "ls_verify_attn.h"
+
+namespace {
+
+using ls::Plan;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];  // 0 = not queried yet; a benign race writes the same value
+int g_cc_major[kMaxDevices];
+
+int device_info(int* sm_count, int* cc_major) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LS_ERR_CUDA;
+  if (dev < kMaxDevices && g_sm_count[dev] > 0) {
+    *sm_count = g_sm_count[dev];
+    *cc_major = g_cc_major[dev];
+    return LS_OK;
+  }
+  int sms = 0, major = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return LS_ERR_CUDA;
+  if (dev < kMaxDevices) {
+    g_cc_major[dev] = major;
+    g_sm_count[dev] = sms;
+  }
+  *sm_count = sms;
+  *cc_major = major;
+  return LS_OK;
+}
+
+int check_dims(const ls_verify_dims* d) {
+  if (d == nullptr) return LS_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1 || d->tree_size < 1 ||
+      d->max_prefix_len < 0)
+    return LS_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return LS_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return LS_ERR_UNSUPPORTED;
+  if (d->tree_size > ls::kMaxTree) return LS_ERR_UNSUPPORTED;
+  // index arithmetic stays in int32 for rows and in size_t for element offsets
+  const long long rows = (long long)d->batch * d->tree_size * d->num_q_heads;
+  if (rows > (1ll << 30)) return LS_ERR_UNSUPPORTED;
+  if (d->cu_seqlens_host != nullptr) {
+    const int32_t* cu = d->cu_seqlens_host;
+    if (cu[0] != 0) return LS_ERR_INVALID_ARG;
+    for (int b = 0; b < d->batch; ++b)
+      if (cu[b + 1] < cu[b]) return LS_ERR_INVALID_ARG;
+  }
+  return LS_OK;
+}
+
+// Chooses the chunk length C (in 128-key blocks) that minimises the estimated time of
+// the prefix kernel: waves of `slots` CTAs, each wave as long as its longest chunk
+// plus a fixed per-chunk cost for loading Q and writing the partial.
+int make_plan(const ls_verify_dims* d, Plan* p) {
+  int rc = check_dims(d);
+  if (rc != LS_OK) return rc;
+  int sms = 0, major = 0;
+  rc = device_info(&sms, &major);
+  if (rc != LS_OK) return rc;
+  if (major != 10) return LS_ERR_UNSUPPORTED;
+
+  Plan q{};
+  q.B = d->batch;
+  q.Hq = d->num_q_heads;
+  q.Hkv = d->num_kv_heads;
+  q.d = d->head_dim;
+  q.T = d->tree_size;
+  q.g = q.Hq / q.Hkv;
+  q.rows = q.T * q.g;
+  q.rg = ls::ceil_div(q.rows, ls::kUnitRows);
+  q.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)q.d);
+  q.scale_log2 = (float)((double)q.scale * 1.4426950408889634074);
+  q.n_combine = q.B * q.T * q.Hkv;
+
+  std::vector<int32_t> blocks(q.B);
+  int32_t max_blocks = 0;
+  for (int b = 0; b < q.B; ++b) {
+    const int32_t L = d->cu_seqlens_host ? d->cu_seqlens_host[b + 1] - d->cu_seqlens_host[b]
+                                         : d->max_prefix_len;
+    blocks[b] = ls::ceil_div(L, ls::kBlockN);
+    if (blocks[b] > max_blocks) max_blocks = blocks[b];
+  }
+  const long long units = (long long)q.Hkv * q.rg;
+  const long long slots = sms;  // one prefix CTA per SM
+  const long long overhead = 2;  // per-chunk cost in blocks (Q load, partial store)
+  int32_t best_C = max_blocks > 0 ? max_blocks : 1;
+  long long best_cost = -1, best_n = 0;
+  for (int32_t C = 1; C <= max_blocks; ++C) {
+    long long n = 0;
+    for (int b = 0; b < q.B; ++b) n += units * ls::ceil_div(blocks[b], C);
+    const long long waves = (n + slots - 1) / slots;
+    const long long cost = waves * (C + overhead);
+    if (best_cost < 0 || cost < best_cost || (cost == best_cost && n < best_n)) {
+      best_cost = cost;
+      best_C = C;
+      best_n = n;
+    }
+  }
+  q.C = best_C;
+  if (d->cu_seqlens_host) {
+    q.uniform_n = -1;
+  } else {
+    q.uniform_n = max_blocks > 0 ? ls::ceil_div(max_blocks, q.C) : 0;
+  }
+  long long n = 0;
+  for (int b = 0; b < q.B; ++b)
+    n += units * (q.uniform_n >= 0 ? q.uniform_n : ls::ceil_div(blocks[b], q.C));
+  if (n > (1ll << 30)) return LS_ERR_UNSUPPORTED;
+  q.n_chunks = (int32_t)n;
+  *p = q;
+  return LS_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
+bool aligned4(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 3u) == 0; }
+
+bool workspace_ok(const void* ws, size_t bytes, const ls::Layout& lay) {
+  return ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 && bytes >= lay.total;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ls_verify_attn_workspace_size(const ls_verify_dims* dims) {
+  Plan p;
+  if (make_plan(dims, &p) != LS_OK) return 0;
+  return (size_t)ls::make_layout(p).total;
+}
+
+int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* prefix_ctas, int32_t* blocks_per_chunk,
+                        int32_t* combine_ctas) {
+  Plan p;
+  const int rc = make_plan(dims, &p);
+  if (rc != LS_OK) return rc;
+  if (prefix_ctas) *prefix_ctas = p.n_chunks;
+  if (blocks_per_chunk) *blocks_per_chunk = p.C;
+  if (combine_ctas) *combine_ctas = p.n_combine;
+  return LS_OK;
+}
+
+int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* cu_seqlens, const ls_verify_dims* dims, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(dims, &p);
+  if (rc != LS_OK) return rc;
+  if (q == nullptr || cu_seqlens == nullptr || !aligned16(q) || !aligned4(cu_seqlens))
+    return LS_ERR_INVALID_ARG;
+  if (p.n_chunks > 0 && (k_cache == nullptr || v_cache == nullptr || !aligned16(k_cache) ||
+                         !aligned16(v_cache)))
+    return LS_ERR_INVALID_ARG;
+  const ls::Layout lay = ls::make_layout(p);
+  if (!workspace_ok(workspace, workspace_bytes, lay)) return LS_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  (void)cudaGetLastError();  // clear a stale, non-sticky error from unrelated work
+  ls::PrefixArgs pa;
+  pa.q = static_cast<const uint16_t*>(q);
+  pa.k_cache = static_cast<const uint16_t*>(k_cache);
+  pa.v_cache = static_cast<const uint16_t*>(v_cache);
+  pa.cu = cu_seqlens;
+  pa.o_part = reinterpret_cast<float*>(ws + lay.o_part);
+  pa.lse_part = reinterpret_cast<float*>(ws + lay.lse_part);
+  pa.chunk_status = reinterpret_cast<uint32_t*>(ws + lay.chunk_status);
+  pa.p = p;
+  if (ls::launch_prefix_simt(pa, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LS_ERR_CUDA;
+  return LS_OK;
+}
+
+int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const void* v_tree,
+                                const int32_t* tree_parent, const int32_t* cu_seqlens, void* out,
+                                float* lse, const ls_verify_dims* dims, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(dims, &p);
+  if (rc != LS_OK) return rc;
+  const void* ptrs16[] = {q, k_tree, v_tree, out};
+  for (const void* x : ptrs16)
+    if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
+  const void* ptrs4[] = {tree_parent, cu_seqlens, lse};
+  for (const void* x : ptrs4)
+    if (x == nullptr || !aligned4(x)) return LS_ERR_INVALID_ARG;
+  const ls::Layout lay = ls::make_layout(p);
+  if (!workspace_ok(workspace, workspace_bytes, lay)) return LS_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  (void)cudaGetLastError();
+  ls::CombineArgs ca;
+  ca.q = static_cast<const uint16_t*>(q);
+  ca.k_tree = static_cast<const uint16_t*>(k_tree);
+  ca.v_tree = static_cast<const uint16_t*>(v_tree);
+  ca.parent = tree_parent;
+  ca.cu = cu_seqlens;
+  ca.o_part = reinterpret_cast<const float*>(ws + lay.o_part);
+  ca.lse_part = reinterpret_cast<const float*>(ws + lay.lse_part);
+  ca.chunk_status = reinterpret_cast<const uint32_t*>(ws + lay.chunk_status);
+  ca.out = static_cast<uint16_t*>(out);
+  ca.lse = lse;
+  ca.status = reinterpret_cast<uint32_t*>(ws + lay.status);
+  ca.p = p;
+  if (ls::launch_tree_combine(ca, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LS_ERR_CUDA;
+  return LS_OK;
+}
+
+int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache, const void* k_tree,
+                   const void* v_tree, const int32_t* tree_parent, const int32_t* cu_seqlens,
+                   void* out, float* lse, const ls_verify_dims* dims, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  // check every argument of both stages before launching the first
+  Plan p;
+  int rc = make_plan(dims, &p);
+  if (rc != LS_OK) return rc;
+  const void* ptrs16[] = {q, k_tree, v_tree, out};
+  for (const void* x : ptrs16)
+    if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
+  const void* ptrs4[] = {tree_parent, cu_seqlens, lse};
+  for (const void* x : ptrs4)
+    if (x == nullptr || !aligned4(x)) return LS_ERR_INVALID_ARG;
+  rc = ls_verify_attn_prefix(q, k_cache, v_cache, cu_seqlens, dims, workspace, workspace_bytes,
+                             stream);
+  if (rc != LS_OK) return rc;
+  return ls_verify_attn_tree_combine(q, k_tree, v_tree, tree_parent, cu_seqlens, out, lse, dims,
+                                     workspace, workspace_bytes, stream);
+}
+
+int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void* stream) {
+  Plan p;
+  int rc = make_plan(dims, &p);
+  if (rc != LS_OK) return rc;
+  if (workspace == nullptr) return LS_ERR_WORKSPACE;
+  const ls::Layout lay = ls::make_layout(p);
+  std::vector<uint32_t> st(p.n_combine);
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LS_ERR_CUDA;
+  if (cudaMemcpy(st.data(), static_cast<const char*>(workspace) + lay.status,
+                 st.size() * sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LS_ERR_CUDA;
+  uint32_t all = 0;
+  for (uint32_t v : st) all |= v;
+  if (all & ls::kErrLengths) return LS_ERR_LENGTHS;
+  if (all & ls::kErrBadTree) return LS_ERR_BAD_TREE;
+  if (all & ls::kErrTimeout) return LS_ERR_TIMEOUT;
+  return LS_OK;
+}
+
+const char* ls_status_string(int status) {
+  switch (status) {
+    case LS_OK: return "ok";
+    case LS_ERR_INVALID_ARG: return "invalid argument";
+    case LS_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case LS_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case LS_ERR_CUDA: return "CUDA launch or copy failed";
+    case LS_ERR_BAD_TREE: return "tree_parent is not a rooted tree with parent[i] < i";
+    case LS_ERR_TIMEOUT: return "a device-side wait timed out";
+    case LS_ERR_LENGTHS: return "device cu_seqlens disagrees with the planned lengths";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

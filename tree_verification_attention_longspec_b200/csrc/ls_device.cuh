@@ -1,0 +1,59 @@
+// Device-side helpers and kernel argument blocks.
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ls_plan.cuh"
+
+namespace ls {
+
+constexpr float kLn2 = 0.693147180559945309417f;
+
+struct PrefixArgs {
+  const uint16_t* q;
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;
+  const int32_t* cu;
+  float* o_part;
+  float* lse_part;
+  uint32_t* chunk_status;
+  Plan p;
+};
+
+struct CombineArgs {
+  const uint16_t* q;
+  const uint16_t* k_tree;
+  const uint16_t* v_tree;
+  const int32_t* parent;
+  const int32_t* cu;
+  const float* o_part;
+  const float* lse_part;
+  const uint32_t* chunk_status;
+  uint16_t* out;
+  float* lse;
+  uint32_t* status;
+  Plan p;
+};
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t bits) {
+  return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace ls
+
+// Launchers (defined in the kernel files, called by the host API).
+namespace ls {
+cudaError_t launch_prefix_simt(const PrefixArgs& a, cudaStream_t stream);
+cudaError_t launch_tree_combine(const CombineArgs& a, cudaStream_t stream);
+}  // namespace ls
