@@ -8,6 +8,19 @@ OUT_ATOL = 1e-2   # max-abs error on bf16 `out` against the fp64 oracle
 LSE_ATOL = 1e-3   # max-abs error on fp32 `lse`
 
 
+def bf16_ulp(x):
+    """Spacing of bf16 numbers at |x| (8 significant bits): 2^(floor(log2|x|) - 7)."""
+    ax = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), np.finfo(np.float64).tiny)
+    return np.exp2(np.floor(np.log2(ax)) - 7)
+
+
+def out_tolerance(ref):
+    """Per-element bound on |out - ref|: 1e-2, except where bf16 itself cannot resolve
+    it. For |ref| >= 2 one bf16 ulp exceeds 2^-7 = 0.0078 and round-to-nearest alone
+    costs half an ulp, so the bound there is one ulp at |ref|."""
+    return np.maximum(OUT_ATOL, bf16_ulp(ref))
+
+
 def to_device(inp, device="cuda:0"):
     import torch
 

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <vector>
 
@@ -173,8 +174,15 @@ int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cach
   pa.lse_part = reinterpret_cast<float*>(ws + lay.lse_part);
   pa.chunk_status = reinterpret_cast<uint32_t*>(ws + lay.chunk_status);
   pa.p = p;
-  if (ls::launch_prefix_simt(pa, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return LS_ERR_CUDA;
+  // rows of the K/V tensors that the TMA descriptors may address (an upper bound is
+  // enough: no block is ever read past its sequence's end)
+  const int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
+                                                : (int64_t)dims->batch * dims->max_prefix_len;
+  const char* impl = getenv("LS_PREFIX_IMPL");
+  const bool simt = impl != nullptr && impl[0] == 's';
+  const cudaError_t e = simt ? ls::launch_prefix_simt(pa, static_cast<cudaStream_t>(stream))
+                             : ls::launch_prefix_tc(pa, kv_rows, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
 }
 
