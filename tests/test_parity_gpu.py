@@ -131,3 +131,15 @@ def test_length_mismatch_reported():
     dev["cu_seqlens"] = torch.from_numpy(short).to("cuda:0")
     _, _, st = run_gpu(inp, dev=dev, op=op)
     assert st == 7                  # LS_ERR_LENGTHS
+
+
+def test_workspace_contents_do_not_matter():
+    """The workspace needs no initialisation: NaN bytes in it (including the slots of
+    empty chunks, which are never written) must not reach the output."""
+    inp = _small(4, 8, 2, 128, 10, [700, 0, 1, 3000], "uniform", seed=8)
+    dev = to_device(inp)
+    op = make_op(inp, host_lengths=False)
+    op.workspace.fill_(0xFF)
+    out, lse, st = run_gpu(inp, dev=dev, op=op)
+    assert st == 0
+    _compare(inp, out, lse)

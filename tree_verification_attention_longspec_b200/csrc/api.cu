@@ -3,7 +3,6 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
-#include <cstdlib>
 #include <cstdint>
 #include <vector>
 
@@ -178,10 +177,7 @@ int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cach
   // enough: no block is ever read past its sequence's end)
   const int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
                                                 : (int64_t)dims->batch * dims->max_prefix_len;
-  const char* impl = getenv("LS_PREFIX_IMPL");
-  const bool simt = impl != nullptr && impl[0] == 's';
-  const cudaError_t e = simt ? ls::launch_prefix_simt(pa, static_cast<cudaStream_t>(stream))
-                             : ls::launch_prefix_tc(pa, kv_rows, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = ls::launch_prefix_tc(pa, kv_rows, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
 }

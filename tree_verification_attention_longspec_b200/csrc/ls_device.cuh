@@ -54,7 +54,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Launchers (defined in the kernel files, called by the host API).
 namespace ls {
-cudaError_t launch_prefix_simt(const PrefixArgs& a, cudaStream_t stream);
 cudaError_t launch_prefix_tc(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream);
 cudaError_t launch_tree_combine(const CombineArgs& a, cudaStream_t stream);
 }  // namespace ls

@@ -2,7 +2,7 @@
 //
 // The prefix ("Cached-Teil") work is cut into chunks. A chunk is one
 // (sequence b, kv head kh, row group rg, key range) and becomes one CTA of the
-// prefix kernel. A row group is 256 query rows of one kv head; the rows of a kv
+// prefix kernel. A row group is 128 query rows of one kv head; the rows of a kv
 // head are its T*g (tree node, head-in-group) pairs, row r = i*g + j.
 // Every chunk of a sequence covers C consecutive 128-key blocks (the last one
 // fewer), so the chunk grid follows from the prefix lengths and C alone, and the
@@ -19,7 +19,7 @@
 namespace ls {
 
 constexpr int kBlockN = 128;       // keys per block of the prefix loop
-constexpr int kUnitRows = 256;     // query rows per prefix chunk (two 128-row MMA tiles)
+constexpr int kUnitRows = 128;     // query rows per prefix chunk (one 128-row MMA tile)
 constexpr int kMaxTree = 128;      // largest supported tree
 
 // device-side status bits (combined into one LS_ERR_* by ls_verify_attn_check)
@@ -30,7 +30,7 @@ constexpr uint32_t kErrTimeout = 4u;
 struct Plan {
   int32_t B, Hq, Hkv, d, T, g;
   int32_t rows;        // T * g query rows per (sequence, kv head)
-  int32_t rg;          // row groups per (sequence, kv head): ceil(rows / 256)
+  int32_t rg;          // row groups per (sequence, kv head): ceil(rows / 128)
   int32_t C;           // 128-key blocks per chunk
   int32_t uniform_n;   // >= 0: chunks per unit for every sequence; -1: from L_b
   int32_t n_chunks;    // prefix CTAs
@@ -104,8 +104,8 @@ LS_HD void sequence_chunks(const Plan& p, const int32_t* cu, int32_t b, int32_t*
 
 // Workspace layout (byte offsets, each 256-aligned).
 struct Layout {
-  uint64_t o_part;        // float [n_chunks][256][d]   prefix partial out, normalised
-  uint64_t lse_part;      // float [n_chunks][256]      prefix partial lse, log2 domain
+  uint64_t o_part;        // float [n_chunks][128][d]   prefix partial out, normalised
+  uint64_t lse_part;      // float [n_chunks][128]      prefix partial lse, log2 domain
   uint64_t chunk_status;  // u32   [n_chunks]
   uint64_t status;        // u32   [n_combine]
   uint64_t total;

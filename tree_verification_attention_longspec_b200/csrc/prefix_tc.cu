@@ -3,27 +3,33 @@
 // LongSpec, gist.science summary, section 2C: the cached prefix is attended with no
 // mask, and it carries most of the work, so it runs on the fastest path. With grouped-
 // query attention the T*g (tree node, head-in-group) rows of one kv head share every
-// key, so the prefix step is a dense contraction: S = Q K^T and O += P V per 128-key
-// block. One CTA handles one chunk: 256 query rows (two 128-row tiles) of one
-// (sequence, kv head) against a range of 128-key blocks, and leaves its partial
-// (out normalised by its own sum, lse in the log2 domain) for the combine kernel.
+// key, so the prefix step is a dense contraction: S = Q K^T and O += P V. One CTA handles
+// one chunk: a 128-row tile of one (sequence, kv head) against a range of 128-key
+// blocks, and leaves its partial (out normalised by its own sum, lse in the log2
+// domain) for the combine kernel.
+//
+// Pipeline. The scores of key block j go to one of two 128-column TMEM buffers (j % 2),
+// so the tensor core computes S(j+1) = Q K(j+1)^T while the softmax works on S(j).
+// The two softmax warpgroups split every block's columns: warpgroup x owns keys
+// [64x, 64x+64) of each block and keeps its own running max m_x, sum l_x and output
+// accumulator O_x += P_x V_x in TMEM, so the halves never wait for each other; they are
+// merged by log-sum-exp once, at the end. P_x (bf16) is written over the scores it came
+// from and read by the PV product straight from TMEM.
 //
 // Warp roles (320 threads, one CTA per SM):
-//   warps 0-3  softmax for tile 0, warps 4-7 softmax for tile 1: one thread per query
-//              row (= TMEM lane). Reads S from TMEM, keeps the running max m and sum l,
-//              writes P (bf16) back over S in TMEM, rescales O in TMEM when m moves up
-//              by more than 2^8, and writes the normalised partial at the end.
-//   warp 8     TMA producer: streams K and V blocks into a ring of shared-memory slots.
-//   warp 9     MMA issuer (one thread): S_t = Q_t K^T (both operands in shared memory)
-//              and O_t += P_t V (P from TMEM, V in shared memory), tcgen05.commit to
-//              mbarriers.
-// A softmax thread never holds a whole score row: it reads S from TMEM twice, once in
-// 32-column chunks for the row maximum and once to turn each chunk into P, which keeps
-// it far below the 168 registers a thread has at 320 threads per SM.
-// TMEM columns: S/P of tile t at 128*t, O of tile t at 256 + D*t (512 allocated).
+//   warps 0-3  softmax of key half 0, warps 4-7 of key half 1: one thread per query
+//              row (= TMEM lane). P is computed against the current m_x in one pass;
+//              only when a block's maximum exceeds m_x by more than 2^8 is m_x raised,
+//              O_x rescaled in TMEM and P recomputed.
+//   warp 8     TMA producer: streams 128-key K and V blocks into a ring of slots.
+//   warp 9     MMA issuer (one thread): S = Q K^T (shared-memory operands, N = 128) and
+//              O_x += P_x V_x (P from TMEM, K = 64, N = d), tcgen05.commit to mbarriers.
+// TMEM columns (512 allocated): score buffer u at 128u, O_x at 256 + d*x.
 // Every wait is bounded: on a timeout the CTA raises an abort flag, all roles drain
 // their in-flight copies and MMAs, TMEM is freed, and the chunk status reports it.
 #include <cudaTypedefs.h>
+
+#include <cstdlib>
 
 #include "ls_device.cuh"
 #include "sm100.cuh"
@@ -36,6 +42,7 @@ constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kMaxSlots = 12;
+constexpr int kHalf = 64;  // keys of a block owned by one softmax warpgroup
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -44,15 +51,16 @@ struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;             // 128 rows x 64 bf16, 128B-swizzled
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // 128 rows x D bf16
-  static constexpr int kSlots = D == 128 ? 5 : 12;
+  static constexpr int kSlots = D == 128 ? 6 : 12;
   static constexpr int kQOff = 0;
-  static constexpr int kSlotOff = 2 * kTileBytes;
+  static constexpr int kSlotOff = kTileBytes;
   static constexpr int kBarOff = kSlotOff + kSlots * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 512 + 1024;   // barriers + alignment slack
+  static constexpr int kSmemBytes = kBarOff + 1024 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
   static_assert(kSlots <= kMaxSlots, "slots");
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct alignas(64) TcParams {
@@ -64,12 +72,14 @@ struct alignas(64) TcParams {
 struct Bars {
   uint64_t full[kMaxSlots];
   uint64_t empty[kMaxSlots];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[2];     // [buffer]: S(j) of buffer j%2 is in TMEM
+  uint64_t p_full[2][2];  // [half][buffer]: P_x(j) is in TMEM
+  uint64_t pv_done[2];    // [half]: O_x += P_x(j) V_x(j) finished
   uint64_t o_full;
   uint32_t tmem_base;
   uint32_t abort;
 };
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 // Waits only on time (used to drain in-flight work after an abort).
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -77,7 +87,28 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait_bounded(bar, parity, &never, kTimeoutNs);
 }
 
-template <int D>
+// P = 2^(s*cs - m) for the 64 scores this thread holds, packed to bf16 pairs; adds the
+// values to (sum0, sum1). EMU of every 4 pairs use the FMA-pipe exponential.
+template <int EMU>
+__device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float m, uint32_t (&pk)[kHalf / 2],
+                                       float& sum0, float& sum1) {
+  const float nm = -m;
+#pragma unroll
+  for (int e = 0; e < kHalf / 2; ++e) {
+    float x0, x1, p0, p1;
+    fma2_bc(x0, x1, s[2 * e], s[2 * e + 1], cs, nm);
+    if ((e & 3) < EMU) {
+      exp2_poly_x2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    add2(sum0, sum1, p0, p1);
+    pk[e] = pack_bf16x2(p0, p1);
+  }
+}
+
+template <int D, int EMU>
 __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_constant__ TcParams P) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -94,7 +125,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
   const int tail_shift = nb * kBlockN - n_keys;  // masked leading columns of the last block
   const int row0 = c.rgi * kUnitRows;
   const int rows_here = min(kUnitRows, p.rows - row0);
-  const int nt = rows_here > 128 ? 2 : 1;
 
   if (nb == 0) {  // empty key range: an empty partial
     if (tid < rows_here) a.lse_part[(size_t)blockIdx.x * kUnitRows + tid] = -INFINITY;
@@ -107,9 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], 128);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bars->s_full[u], 1);
+      mbar_init(&bars->p_full[0][u], 128);
+      mbar_init(&bars->p_full[1][u], 128);
+      mbar_init(&bars->pv_done[u], 1);
     }
     mbar_init(&bars->o_full, 1);
     bars->abort = 0u;
@@ -164,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
     // ------------------------------------------------------------------ load Q (warps 0-7)
     if (warp < 8) {
       const int chunks_per_row = D / 8;  // 16-byte chunks
-      const int total = nt * 128 * chunks_per_row;
+      const int total = 128 * chunks_per_row;
       for (int idx = tid; idx < total; idx += 256) {
         const int r = idx / chunks_per_row, ch = idx % chunks_per_row;
         const int rg = row0 + r;
@@ -174,8 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
           const uint16_t* src = a.q + ((size_t)(c.b * p.T + i) * p.Hq + c.kh * p.g + jh) * D + ch * 8;
           v = *reinterpret_cast<const uint4*>(src);
         }
-        const int t = r >> 7, rr = r & 127, pn = ch >> 3, cc = ch & 7;
-        uint8_t* dst = smem + C::kQOff + t * C::kTileBytes + pn * C::kPanelBytes + rr * 128 + ((cc ^ (rr & 7)) << 4);
+        const int pn = ch >> 3, cc = ch & 7;
+        uint8_t* dst = smem + C::kQOff + pn * C::kPanelBytes + r * 128 + ((cc ^ (r & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = v;
       }
       fence_proxy_async_smem();
@@ -185,54 +217,70 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
 
     if (warp == kMmaWarp) {
       if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, false);
+        // -------------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc_qk = umma_idesc_bf16(128, kBlockN, false);
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, true);
         const uint32_t q_base = smem_u32(smem + C::kQOff);
         const uint32_t slot_base = smem_u32(smem + C::kSlotOff);
-        bool ok = true;
-        for (int j = 0; j <= nb && ok; ++j) {
-          const int sk = (2 * j) % C::kSlots, uk = (2 * j) / C::kSlots;
-          const int sv = (2 * j - 1 + 2 * C::kSlots) % C::kSlots, uv = (2 * j - 1) / C::kSlots;
-          if (j < nb) {
-            ok = mbar_wait_bounded(&bars->full[sk], uk & 1, abort, kTimeoutNs);
+        // K block j is sequence 2j of the slot ring, V block j is sequence 2j+1
+        auto wait_full = [&](int seq) {
+          return mbar_wait_bounded(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1, abort, kTimeoutNs);
+        };
+        // S(j) = Q K(j)^T into score buffer j%2
+        auto issue_qk = [&](int j) {
+          const uint32_t kaddr = slot_base + ((2 * j) % C::kSlots) * C::kTileBytes;
+          const uint32_t tS = tbase + C::kColS + (j & 1) * kBlockN;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+            umma_ss(tS, umma_sdesc_sw128(q_base + off, 16, 1024), umma_sdesc_sw128(kaddr + off, 16, 1024),
+                    idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bars->s_full[j & 1]);
+        };
+        // O_x += P_x(j) V_x(j): K = 64 keys of half x, P from TMEM, V rows of that half
+        auto issue_pv = [&](int x, int j) {
+          const uint32_t vaddr = slot_base + ((2 * j + 1) % C::kSlots) * C::kTileBytes + x * (kHalf * 128);
+          const uint32_t tP = tbase + C::kColS + (j & 1) * kBlockN + x * kHalf;
+          const uint32_t tO = tbase + C::kColO + x * D;
+#pragma unroll
+          for (int kk = 0; kk < kHalf / 16; ++kk)
+            umma_ts(tO, tP + kk * 8, umma_sdesc_sw128(vaddr + kk * 2048, C::kPanelBytes, 1024), idesc_pv,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars->pv_done[x]);
+        };
+        bool ok = wait_full(0);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_qk(0);
+          umma_commit(&bars->empty[0]);
+          if (nb > 1) {
+            ok = wait_full(2);
+            if (ok) {
+              tc_fence_after_sync();
+              issue_qk(1);
+              umma_commit(&bars->empty[2 % C::kSlots]);
+            }
+          }
+        }
+        for (int j = 0; j < nb && ok; ++j) {
+          ok = wait_full(2 * j + 1);  // V block j
+          for (int x = 0; x < 2 && ok; ++x) {
+            ok = mbar_wait_bounded(&bars->p_full[x][j & 1], (j >> 1) & 1, abort, kTimeoutNs);
             if (!ok) break;
             tc_fence_after_sync();
-          }
-          for (int t = 0; t < nt; ++t) {
-            if (j > 0) {
-              // O_t += P_t(j-1) V(j-1)
-              if (t == 0) {
-                ok = mbar_wait_bounded(&bars->full[sv], uv & 1, abort, kTimeoutNs);
-                if (!ok) break;
-              }
-              ok = mbar_wait_bounded(&bars->p_full[t], (j - 1) & 1, abort, kTimeoutNs);
-              if (!ok) break;
-              tc_fence_after_sync();
-              const uint32_t vaddr = slot_base + sv * C::kTileBytes;
-              const uint32_t tP = tbase + C::kColS + t * 128;
-              const uint32_t tO = tbase + C::kColO + t * D;
-#pragma unroll
-              for (int kk = 0; kk < kBlockN / 16; ++kk)
-                umma_ts(tO, tP + kk * 8, umma_sdesc_sw128(vaddr + kk * 2048, C::kPanelBytes, 1024), idesc_pv,
-                        (j > 1 || kk > 0) ? 1u : 0u);
-            }
-            if (j < nb) {
-              // S_t = Q_t K(j)^T
-              const uint32_t kaddr = slot_base + sk * C::kTileBytes;
-              const uint32_t qaddr = q_base + t * C::kTileBytes;
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                umma_ss(tbase + C::kColS + t * 128, umma_sdesc_sw128(qaddr + off, 16, 1024),
-                        umma_sdesc_sw128(kaddr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(&bars->s_full[t]);
-            }
+            issue_pv(x, j);
           }
           if (!ok) break;
-          if (j < nb) umma_commit(&bars->empty[sk]);
-          if (j > 0) umma_commit(&bars->empty[sv]);
+          umma_commit(&bars->empty[(2 * j + 1) % C::kSlots]);
+          if (j + 2 < nb) {
+            // S(j+2) reuses buffer j%2: issued after both halves of P(j) have been read
+            ok = wait_full(2 * (j + 2));
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_qk(j + 2);
+            umma_commit(&bars->empty[(2 * (j + 2)) % C::kSlots]);
+          }
         }
         umma_commit(&bars->o_full);
         drain_wait(&bars->o_full, 0);
@@ -240,98 +288,132 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
       __syncwarp();
     } else {
       // ---------------------------------------------------------------- softmax / epilogue
-      const int t = warp >> 2;
-      if (t < nt) {
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tbase + lane_base + C::kColS + t * 128;
-        const uint32_t tO = tbase + lane_base + C::kColO + t * D;
-        const float cs = p.scale_log2;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int j = 0; j < nb; ++j) {
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], j & 1, abort, kTimeoutNs));
-          if (!ok) break;
-          const int shift = j == nb - 1 ? tail_shift : 0;
-          tc_fence_after_sync();
-          // pass 1: row maximum of the raw scores (masked leading columns excluded)
-          float mx = -INFINITY;
+      const int x = warp >> 2;  // key half
+      const int row = (warp & 3) * 32 + lane;
+      const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t tS0 = tbase + lane_base + C::kColS + x * kHalf;
+      const uint32_t tOx = tbase + lane_base + C::kColO + x * D;
+      const float cs = p.scale_log2;
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nb; ++j) {
+        const int u = j & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[u], (j >> 1) & 1, abort, kTimeoutNs));
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint32_t tS = tS0 + u * kBlockN;
+        float s[kHalf];
+        {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int q4 = 0; q4 < kBlockN / 32; ++q4) {
-            uint32_t r[32];
-            tmem_ld32(tS + q4 * 32, r);
-            tmem_wait_ld();
-            float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const bool k0 = q4 * 32 + e >= shift, k1 = q4 * 32 + e + 1 >= shift;
-              m0 = fmaxf(m0, k0 ? __uint_as_float(r[e]) : -INFINITY);
-              m1 = fmaxf(m1, k1 ? __uint_as_float(r[e + 1]) : -INFINITY);
-            }
-            mx = fmaxf(mx, fmaxf(m0, m1));
+          for (int e = 0; e < 32; ++e) {
+            s[e] = __uint_as_float(r0[e]);
+            s[32 + e] = __uint_as_float(r1[e]);
           }
-          const float m_new = fmaxf(m, mx * cs);
-          const bool need = m_new > m + kRescaleThreshold;
-          if (j > 0 && __any_sync(0xffffffffu, need)) {
-            const float f = need ? ex2_approx(m - m_new) : 1.f;
+        }
+        // the sequence's last block: columns before tail_shift belong to earlier keys
+        const int shift = j == nb - 1 ? tail_shift - x * kHalf : 0;
+        if (shift > 0) {
+#pragma unroll
+          for (int e = 0; e < kHalf; ++e)
+            if (e < shift) s[e] = -INFINITY;
+        }
+        float mx;
+        {
+          float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+          for (int e = 4; e < kHalf; e += 8) {
+            m0 = fmax3(m0, s[e], s[e + 1]);
+            m1 = fmax3(m1, s[e + 2], s[e + 3]);
+            m2 = fmax3(m2, s[e + 4], s[e + 5]);
+            m3 = fmax3(m3, s[e + 6], s[e + 7]);
+          }
+          mx = fmax3(m0, m1, fmaxf(m2, m3)) * cs;  // -inf if the whole half is masked
+        }
+        uint32_t pk[kHalf / 2];
+        float sum0 = 0.f, sum1 = 0.f;
+        const bool raise = mx > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, raise)) {
+          // the maximum moved up: rescale what O_x and l hold (once the previous PV has
+          // landed) and compute P against the new maximum
+          const float m_new = raise ? mx : m;
+          if (j > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[x], (j - 1) & 1, abort, kTimeoutNs));
+            if (!ok) break;
+            tc_fence_after_sync();
+            // f = 1 where m is unchanged; 0 where nothing was accumulated yet (m = -inf)
+            const float f = m == m_new ? 1.f : ex2_approx(m - m_new);
 #pragma unroll
             for (int q4 = 0; q4 < D / 32; ++q4) {
               uint32_t r[32];
-              tmem_ld32(tO + q4 * 32, r);
+              tmem_ld32(tOx + q4 * 32, r);
               tmem_wait_ld();
 #pragma unroll
               for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-              tmem_st32(tO + q4 * 32, r);
+              tmem_st32(tOx + q4 * 32, r);
             }
             l *= f;
           }
-          if (need) m = m_new;
-          const float nm = -m;
-          // pass 2: P = 2^(s*scale*log2e - m) as bf16, written over the part of S already read
-          float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-          for (int q4 = 0; q4 < kBlockN / 32; ++q4) {
-            uint32_t r[32];
-            tmem_ld32(tS + q4 * 32, r);
-            tmem_wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const bool k0 = q4 * 32 + 2 * e >= shift, k1 = q4 * 32 + 2 * e + 1 >= shift;
-              const float p0 = k0 ? ex2_approx(fmaf(__uint_as_float(r[2 * e]), cs, nm)) : 0.f;
-              const float p1 = k1 ? ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), cs, nm)) : 0.f;
-              sum0 += p0;
-              sum1 += p1;
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(tS + q4 * 16, pk);
-          }
-          l += sum0 + sum1;
-          tmem_wait_st();
-          tc_fence_before_sync();
-          mbar_arrive(&bars->p_full[t]);
+          m = m_new;
+          make_p<0>(s, cs, m == -INFINITY ? 0.f : m, pk, sum0, sum1);
+        } else if (shift > 0 || m == -INFINITY) {
+          // masked columns (-inf) stay on the MUFU path; while nothing has been seen yet
+          // (m = -inf, everything so far masked) every P is 0
+          make_p<0>(s, cs, m == -INFINITY ? 0.f : m, pk, sum0, sum1);
+        } else {
+          make_p<EMU>(s, cs, m, pk, sum0, sum1);
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full, 0, abort, kTimeoutNs));
-        if (ok) {
-          tc_fence_after_sync();
-          const int r_local = t * 128 + (warp & 3) * 32 + lane;
-          const bool valid = r_local < rows_here;
-          const float inv = 1.f / l;
-          float* dst = a.o_part + ((size_t)blockIdx.x * kUnitRows + r_local) * D;
+        l += sum0 + sum1;
+        tmem_st32(tS, pk);
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(&bars->p_full[x][u]);
+      }
+      // -------------------------------------------------------------- epilogue
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full, 0, abort, kTimeoutNs));
+      // every MMA has finished (o_full), so the Q tile's shared memory is free: it carries
+      // both halves' (m, l) of every row to the other warpgroup
+      float* xm = reinterpret_cast<float*>(smem + C::kQOff);  // [2][128]
+      float* xl = xm + 256;                                   // [2][128]
+      xm[x * 128 + row] = ok ? m : -INFINITY;
+      xl[x * 128 + row] = ok ? l : 0.f;
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      if (ok) {
+        tc_fence_after_sync();
+        const float ma = xm[row], mb = xm[128 + row];
+        const float M = fmaxf(ma, mb);
+        const float wa = ma == -INFINITY ? 0.f : ex2_approx(ma - M);
+        const float wb = mb == -INFINITY ? 0.f : ex2_approx(mb - M);
+        const float Ls = wa * xl[row] + wb * xl[128 + row];
+        const float inv = 1.f / Ls;
+        const float ca = wa * inv, cb = wb * inv;
+        const bool valid = row < rows_here;
+        // this warpgroup writes output columns [x*D/2, (x+1)*D/2) of its rows
+        float* dst = a.o_part + ((size_t)blockIdx.x * kUnitRows + row) * D + x * (D / 2);
+        const uint32_t tOa = tbase + lane_base + C::kColO + x * (D / 2);
+        const uint32_t tOb = tOa + D;
 #pragma unroll
-          for (int q4 = 0; q4 < D / 32; ++q4) {
-            uint32_t r[32];
-            tmem_ld32(tO + q4 * 32, r);
-            tmem_wait_ld();
-            if (valid) {
+        for (int q4 = 0; q4 < D / 64; ++q4) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tOa + q4 * 32, ra);
+          tmem_ld32(tOb + q4 * 32, rb);
+          tmem_wait_ld();
+          if (valid) {
 #pragma unroll
-              for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(dst + q4 * 32 + e) =
-                    make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
-                                __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+            for (int e = 0; e < 32; e += 4) {
+              float4 v;
+              v.x = fmaf(ca, __uint_as_float(ra[e]), cb * __uint_as_float(rb[e]));
+              v.y = fmaf(ca, __uint_as_float(ra[e + 1]), cb * __uint_as_float(rb[e + 1]));
+              v.z = fmaf(ca, __uint_as_float(ra[e + 2]), cb * __uint_as_float(rb[e + 2]));
+              v.w = fmaf(ca, __uint_as_float(ra[e + 3]), cb * __uint_as_float(rb[e + 3]));
+              *reinterpret_cast<float4*>(dst + q4 * 32 + e) = v;
             }
           }
-          if (valid) a.lse_part[(size_t)blockIdx.x * kUnitRows + r_local] = m + log2f(l);
         }
+        if (valid && x == 0) a.lse_part[(size_t)blockIdx.x * kUnitRows + row] = M + log2f(Ls);
       }
     }
   }
@@ -371,7 +453,7 @@ bool make_kv_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t row
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int EMU>
 cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) {
   TcParams P;
   P.a = a;
@@ -379,9 +461,16 @@ cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) 
       !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows))
     return cudaErrorInvalidValue;
   const int smem = Cfg<D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(prefix_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  prefix_tc_kernel<D><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
+  // opt in to the large shared-memory carve-out once per device
+  static bool configured[64] = {};  // per template instance
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(prefix_tc_kernel<D, EMU>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) configured[dev] = true;
+  }
+  prefix_tc_kernel<D, EMU><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
   return cudaGetLastError();
 }
 
@@ -389,7 +478,14 @@ cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) 
 
 cudaError_t launch_prefix_tc(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) {
   if (a.p.n_chunks == 0) return cudaSuccess;
-  return a.p.d == 64 ? launch_d<64>(a, kv_rows, stream) : launch_d<128>(a, kv_rows, stream);
+  const char* env = getenv("LS_EMU");
+  const int emu = env ? atoi(env) : 0;
+  if (a.p.d == 64) return launch_d<64, 0>(a, kv_rows, stream);
+  switch (emu) {
+    case 1: return launch_d<128, 1>(a, kv_rows, stream);
+    case 2: return launch_d<128, 2>(a, kv_rows, stream);
+    default: return launch_d<128, 0>(a, kv_rows, stream);
+  }
 }
 
 }  // namespace ls

@@ -196,11 +196,92 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
+      "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
+      "%56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
+        "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+}
+
 // ----------------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two fp32 lanes at once: (d0, d1) = (a0*b + c, a1*b + c)
+__device__ __forceinline__ void fma2_bc(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 rs, ra;\n\t"
+      "mov.b64 rs, {%0, %1};\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "add.rn.f32x2 rs, rs, ra;\n\t"
+      "mov.b64 {%0, %1}, rs;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+
+// 2^x for two values at once on the FMA pipe instead of the MUFU unit.
+// Cody-Waite range reduction: n = round(x) by adding and subtracting 1.5*2^23,
+// f = x - n in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error
+// below 7.5e-5, coefficients from exp2_poly_fit.py); 2^n by adding n to the exponent
+// field (the low bits of x + 1.5*2^23 hold n, so (bits << 23) is n << 23). x is
+// clamped at -125 so the result stays a normal number; x must be at most 127.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, float& p1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  uint32_t t0, t1, q0, q1;
+  asm("{\n\t.reg .b64 x, t, n, f, q, m, mm, c0, c1, c2, c3;\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "mov.b64 m, {%6, %6};\n\t"
+      "mov.b64 mm, {%7, %7};\n\t"
+      "add.rn.f32x2 t, x, m;\n\t"
+      "add.rn.f32x2 n, t, mm;\n\t"
+      "sub.rn.f32x2 f, x, n;\n\t"
+      "mov.b64 c3, {%11, %11};\n\t"
+      "mov.b64 c2, {%10, %10};\n\t"
+      "mov.b64 c1, {%9, %9};\n\t"
+      "mov.b64 c0, {%8, %8};\n\t"
+      "fma.rn.f32x2 q, c3, f, c2;\n\t"
+      "fma.rn.f32x2 q, q, f, c1;\n\t"
+      "fma.rn.f32x2 q, q, f, c0;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t"
+      "mov.b64 {%2, %3}, q;\n\t}"
+      : "=r"(t0), "=r"(t1), "=r"(q0), "=r"(q1)
+      : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(-12582912.0f), "f"(9.999280572e-01f),
+        "f"(6.932609677e-01f), "f"(2.426111251e-01f), "f"(5.517166853e-02f));
+  p0 = __uint_as_float(q0 + (t0 << 23));
+  p1 = __uint_as_float(q1 + (t1 << 23));
 }
 
 // (lo, hi) -> packed bf16x2 with `lo` in the low half, round to nearest even.
