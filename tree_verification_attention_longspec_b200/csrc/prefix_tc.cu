@@ -24,6 +24,9 @@
 //   warp 8     TMA producer: streams 128-key K and V blocks into a ring of slots.
 //   warp 9     MMA issuer (one thread): S = Q K^T (shared-memory operands, N = 128) and
 //              O_x += P_x V_x (P from TMEM, K = 64, N = d), tcgen05.commit to mbarriers.
+//              It waits once per block and then issues the block's 16 MMAs back to back:
+//              MMA issue is throttled to the tensor pipe's pace, so every pause of this
+//              thread is idle tensor time.
 // TMEM columns (512 allocated): score buffer u at 128u, O_x at 256 + d*x.
 // Every wait is bounded: on a timeout the CTA raises an abort flag, all roles drain
 // their in-flight copies and MMAs, TMEM is freed, and the chunk status reports it.
@@ -74,7 +77,7 @@ struct Bars {
   uint64_t empty[kMaxSlots];
   uint64_t s_full[2];     // [buffer]: S(j) of buffer j%2 is in TMEM
   uint64_t p_full[2][2];  // [half][buffer]: P_x(j) is in TMEM
-  uint64_t pv_done[2];    // [half]: O_x += P_x(j) V_x(j) finished
+  uint64_t pv_last;       // O += P(nb-2) V(nb-2) finished (lets the last block rescale O)
   uint64_t o_full;
   uint32_t tmem_base;
   uint32_t abort;
@@ -141,9 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
       mbar_init(&bars->s_full[u], 1);
       mbar_init(&bars->p_full[0][u], 128);
       mbar_init(&bars->p_full[1][u], 128);
-      mbar_init(&bars->pv_done[u], 1);
     }
     mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->pv_last, 1);
     bars->abort = 0u;
     fence_mbar_init();
   }
@@ -160,6 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
   tc_fence_after_sync();
   const uint32_t tbase = bars->tmem_base;
   volatile uint32_t* abort = &bars->abort;
+  // the tree/combine kernel may start its own prologue now; it waits for this grid's
+  // results before it reads them
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
@@ -220,67 +226,85 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
         // -------------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_qk = umma_idesc_bf16(128, kBlockN, false);
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, true);
-        const uint32_t q_base = smem_u32(smem + C::kQOff);
-        const uint32_t slot_base = smem_u32(smem + C::kSlotOff);
+        // A descriptor differs from another of the same kind only in its start-address
+        // field (address >> 4 in the low 14 bits; shared addresses stay below 256 KB, so
+        // adding an offset never carries out of it): build the bases once, add offsets.
+        const uint64_t dq = umma_sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+        const uint64_t dk0 = umma_sdesc_sw128(smem_u32(smem + C::kSlotOff), 16, 1024);
+        const uint64_t dv0 = umma_sdesc_sw128(smem_u32(smem + C::kSlotOff), C::kPanelBytes, 1024);
+        constexpr uint32_t kTile16 = C::kTileBytes >> 4, kPanel16 = C::kPanelBytes >> 4;
         // K block j is sequence 2j of the slot ring, V block j is sequence 2j+1
         auto wait_full = [&](int seq) {
           return mbar_wait_bounded(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1, abort, kTimeoutNs);
         };
-        // S(j) = Q K(j)^T into score buffer j%2
-        auto issue_qk = [&](int j) {
-          const uint32_t kaddr = slot_base + ((2 * j) % C::kSlots) * C::kTileBytes;
+        // S(j) = Q K(j)^T into score buffer j%2; K(j) sits in ring slot `slot`
+        auto issue_qk = [&](int j, int slot) {
+          const uint64_t dk = dk0 + (uint64_t)(slot * kTile16);
           const uint32_t tS = tbase + C::kColS + (j & 1) * kBlockN;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-            umma_ss(tS, umma_sdesc_sw128(q_base + off, 16, 1024), umma_sdesc_sw128(kaddr + off, 16, 1024),
-                    idesc_qk, kk > 0 ? 1u : 0u);
+            const uint32_t off = (kk >> 2) * kPanel16 + (kk & 3) * 2;  // 16-byte units
+            umma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
           }
           umma_commit(&bars->s_full[j & 1]);
         };
-        // O_x += P_x(j) V_x(j): K = 64 keys of half x, P from TMEM, V rows of that half
-        auto issue_pv = [&](int x, int j) {
-          const uint32_t vaddr = slot_base + ((2 * j + 1) % C::kSlots) * C::kTileBytes + x * (kHalf * 128);
+        // O_x += P_x(j) V_x(j): K = 64 keys of half x, P from TMEM, V rows of that half;
+        // V(j) sits in ring slot `slot`
+        auto issue_pv = [&](int x, int j, int slot) {
+          const uint64_t dv = dv0 + (uint64_t)(slot * kTile16 + x * (kHalf * 128 / 16));
           const uint32_t tP = tbase + C::kColS + (j & 1) * kBlockN + x * kHalf;
           const uint32_t tO = tbase + C::kColO + x * D;
 #pragma unroll
           for (int kk = 0; kk < kHalf / 16; ++kk)
-            umma_ts(tO, tP + kk * 8, umma_sdesc_sw128(vaddr + kk * 2048, C::kPanelBytes, 1024), idesc_pv,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars->pv_done[x]);
+            umma_ts(tO, tP + kk * 8, dv + kk * (2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         };
         bool ok = wait_full(0);
         if (ok) {
           tc_fence_after_sync();
-          issue_qk(0);
+          issue_qk(0, 0);
           umma_commit(&bars->empty[0]);
           if (nb > 1) {
             ok = wait_full(2);
             if (ok) {
               tc_fence_after_sync();
-              issue_qk(1);
+              issue_qk(1, 2 % C::kSlots);
               umma_commit(&bars->empty[2 % C::kSlots]);
             }
           }
         }
+        // One wait point per block, then all of the block's MMAs back to back:
+        // O_x += P_x(j) V_x(j) for both halves, then S(j+2) into buffer j%2 (whose P(j)
+        // has just been consumed). Three commits per block: V(j)'s slot, S(j+2) and
+        // K(j+2)'s slot. Slot indices and phases advance incrementally (V(j) is sequence
+        // 2j+1, K(j+2) is sequence 2j+4 of the ring).
+        int sv = 1 % C::kSlots, uv = 1 / C::kSlots;  // V(j): slot and use count parity
+        int sk = 4 % C::kSlots, uk = 4 / C::kSlots;  // K(j+2)
         for (int j = 0; j < nb && ok; ++j) {
-          ok = wait_full(2 * j + 1);  // V block j
-          for (int x = 0; x < 2 && ok; ++x) {
-            ok = mbar_wait_bounded(&bars->p_full[x][j & 1], (j >> 1) & 1, abort, kTimeoutNs);
+          const bool more = j + 2 < nb;
+          uint64_t* bk = more ? &bars->full[sk] : &bars->full[sv];  // no K(j+2): test V twice
+          const uint32_t pk = more ? (uk & 1) : (uv & 1);
+          const uint32_t pp = (j >> 1) & 1;
+          if (!mbar_try_wait4(&bars->full[sv], uv & 1, bk, pk, &bars->p_full[0][j & 1], pp,
+                              &bars->p_full[1][j & 1], pp)) {
+            ok = mbar_wait_bounded(&bars->full[sv], uv & 1, abort, kTimeoutNs) &&
+                 mbar_wait_bounded(bk, pk, abort, kTimeoutNs) &&
+                 mbar_wait_bounded(&bars->p_full[0][j & 1], pp, abort, kTimeoutNs) &&
+                 mbar_wait_bounded(&bars->p_full[1][j & 1], pp, abort, kTimeoutNs);
             if (!ok) break;
-            tc_fence_after_sync();
-            issue_pv(x, j);
           }
-          if (!ok) break;
-          umma_commit(&bars->empty[(2 * j + 1) % C::kSlots]);
-          if (j + 2 < nb) {
-            // S(j+2) reuses buffer j%2: issued after both halves of P(j) have been read
-            ok = wait_full(2 * (j + 2));
-            if (!ok) break;
-            tc_fence_after_sync();
-            issue_qk(j + 2);
-            umma_commit(&bars->empty[(2 * (j + 2)) % C::kSlots]);
+          tc_fence_after_sync();
+          issue_pv(0, j, sv);
+          issue_pv(1, j, sv);
+          umma_commit(&bars->empty[sv]);
+          if (j == nb - 2) umma_commit(&bars->pv_last);
+          if (more) {
+            issue_qk(j + 2, sk);
+            umma_commit(&bars->empty[sk]);
           }
+          sv += 2;
+          if (sv >= C::kSlots) { sv -= C::kSlots; uv ^= 1; }
+          sk += 2;
+          if (sk >= C::kSlots) { sk -= C::kSlots; uk ^= 1; }
         }
         umma_commit(&bars->o_full);
         drain_wait(&bars->o_full, 0);
@@ -341,7 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
           // landed) and compute P against the new maximum
           const float m_new = raise ? mx : m;
           if (j > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->pv_done[x], (j - 1) & 1, abort, kTimeoutNs));
+            // O_x must hold all of PV(j-1) before it is rescaled. QK(j+1) was issued after
+            // PV(j-1), so S(j+1) being ready implies it; the last block has no S(j+1) and
+            // waits for the commit issued after PV(nb-2) instead.
+            ok = __all_sync(0xffffffffu, j + 1 < nb ? mbar_wait_bounded(&bars->s_full[(j + 1) & 1], ((j + 1) >> 1) & 1,
+                                                                        abort, kTimeoutNs)
+                                                    : mbar_wait_bounded(&bars->pv_last, 0, abort, kTimeoutNs));
             if (!ok) break;
             tc_fence_after_sync();
             // f = 1 where m is unchanged; 0 where nothing was accumulated yet (m = -inf)
@@ -358,10 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
             l *= f;
           }
           m = m_new;
-          make_p<0>(s, cs, m == -INFINITY ? 0.f : m, pk, sum0, sum1);
-        } else if (shift > 0 || m == -INFINITY) {
-          // masked columns (-inf) stay on the MUFU path; while nothing has been seen yet
-          // (m = -inf, everything so far masked) every P is 0
+        }
+        // masked columns (-inf) and the rare blocks above take the MUFU-only path; while
+        // nothing has been seen yet (m = -inf, everything so far masked) every P is 0
+        if (EMU == 0 || shift > 0 || m == -INFINITY || __any_sync(0xffffffffu, raise)) {
           make_p<0>(s, cs, m == -INFINITY ? 0.f : m, pk, sum0, sum1);
         } else {
           make_p<EMU>(s, cs, m, pk, sum0, sum1);

@@ -50,6 +50,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Tests four barrier phases at once (the four probes are independent, so they are in
+// flight together); true if all four have completed.
+__device__ __forceinline__ bool mbar_try_wait4(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                               uint32_t p2, uint64_t* b3, uint32_t p3) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q0, q1, q2, q3;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q0, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q1, [%3], %4;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q2, [%5], %6;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q3, [%7], %8;\n\t"
+      "and.pred q0, q0, q1;\n\t"
+      "and.pred q2, q2, q3;\n\t"
+      "and.pred q0, q0, q2;\n\t"
+      "selp.u32 %0, 1, 0, q0;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1), "r"(smem_u32(b2)), "r"(p2), "r"(smem_u32(b3)),
+        "r"(p3)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete. Gives up after
 // `timeout_ns` of global time, or as soon as another thread has raised *abort, and
 // then returns false (raising *abort itself on a timeout). Never spins forever.

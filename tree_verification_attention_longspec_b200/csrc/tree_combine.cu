@@ -15,10 +15,11 @@
 //      every other node's parent lies in [0, c), so the walk ends after at most i+1
 //      steps); then all threads stage the visible nodes' keys and values in shared
 //      memory;
-//   3. each warp issues the loads of its row's prefix partials (every lane one chunk's
-//      lse, up to 16 chunk outputs in flight), runs the online softmax over the staged
-//      tree keys while they arrive, then merges everything by log-sum-exp and writes
-//      bf16 `out` and the natural-log `lse`.
+//   3. each warp runs the online softmax over the staged tree keys of its head, then
+//      waits for the prefix kernel (this kernel is launched as its programmatic
+//      dependent, so rounds 1-3 overlap the prefix kernel's tail), loads its row's prefix
+//      partials (every lane one chunk's lse, up to 16 chunk outputs in flight), merges
+//      everything by log-sum-exp and writes bf16 `out` and the natural-log `lse`.
 #include "ls_device.cuh"
 
 namespace ls {
@@ -93,7 +94,8 @@ __global__ void __launch_bounds__(256) tree_combine_kernel(CombineArgs a) {
   }
   __syncthreads();
 
-  // ---- round 3
+  // ---- round 3: tree part per head, then (once the prefix kernel has finished) its
+  // prefix partials
   uint32_t err_w = 0;
   for (int j = warp; j < p.g; j += nwarps) {
     const size_t row = (size_t)tok * p.Hq + kh * p.g + j;
@@ -131,8 +133,6 @@ __global__ void __launch_bounds__(256) tree_combine_kernel(CombineArgs a) {
         }
       }
     };
-    issue(0);
-
     float qv[E], o[E];
     if (j == warp) {
 #pragma unroll
@@ -143,22 +143,51 @@ __global__ void __launch_bounds__(256) tree_combine_kernel(CombineArgs a) {
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] = 0.f;
-    // tree part: online softmax over node i and its ancestors (log2 domain)
+    // tree part: online softmax over node i and its ancestors (log2 domain), four keys
+    // at a time so that their warp reductions overlap
     float m = -INFINITY, l = 0.f;
-    for (int x = 0; x < na; ++x) {
-      const uint16_t* kr = kt_s + (size_t)x * D + lane * E;
-      float dot = 0.f;
+    for (int x0 = 0; x0 < na; x0 += 4) {
+      float d4[4];
 #pragma unroll
-      for (int e = 0; e < E; ++e) dot = fmaf(qv[e], bf16_to_f32(kr[e]), dot);
-      const float s = warp_sum(dot) * p.scale_log2;
-      const float mn = fmaxf(m, s);
-      const float corr = exp2f(m - mn), w = exp2f(s - mn);
-      l = l * corr + w;
-      const uint16_t* vr = vt_s + (size_t)x * D + lane * E;
+      for (int u = 0; u < 4; ++u) {
+        d4[u] = 0.f;
+        if (x0 + u < na) {
+          const uint16_t* kr = kt_s + (size_t)(x0 + u) * D + lane * E;
 #pragma unroll
-      for (int e = 0; e < E; ++e) o[e] = fmaf(w, bf16_to_f32(vr[e]), o[e] * corr);
+          for (int e = 0; e < E; ++e) d4[u] = fmaf(qv[e], bf16_to_f32(kr[e]), d4[u]);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) d4[u] += __shfl_xor_sync(0xffffffffu, d4[u], off);
+      }
+      float mn = m;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        d4[u] = x0 + u < na ? d4[u] * p.scale_log2 : -INFINITY;
+        mn = fmaxf(mn, d4[u]);
+      }
+      const float corr = exp2f(m - mn);  // m = -inf on the first group: 0
+      l *= corr;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] *= corr;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (x0 + u < na) {
+          const float w = exp2f(d4[u] - mn);
+          l += w;
+          const uint16_t* vr = vt_s + (size_t)(x0 + u) * D + lane * E;
+#pragma unroll
+          for (int e = 0; e < E; ++e) o[e] = fmaf(w, bf16_to_f32(vr[e]), o[e]);
+        }
+      }
       m = mn;
     }
+    // The prefix kernel may still be running (programmatic dependent launch): wait for
+    // it, then fold in its partials. The tree part above overlapped its tail.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    issue(0);
     // merge: the tree part is (lse M, normalised out acc); each chunk adds (lx, ov)
     float M = m + log2f(l);
     float acc[E];
@@ -212,8 +241,20 @@ cudaError_t launch_d(const CombineArgs& a, cudaStream_t stream) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  tree_combine_kernel<D><<<grid, 32 * warps, smem, stream>>>(a);
-  return cudaGetLastError();
+  // launched as a programmatic dependent of the prefix kernel: its first two rounds
+  // (the tree) overlap the prefix kernel's tail; it waits for the prefix partials with
+  // griddepcontrol.wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(32 * warps);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tree_combine_kernel<D>, a);
 }
 
 }  // namespace
