@@ -137,6 +137,34 @@ LS_API int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const 
                                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * ls_verify_attn without a workspace argument, for callers that cannot allocate device
+ * memory (the LongSpec pages have no counterpart: this is an interface convenience).
+ *
+ * ls_verify_attn needs caller-provided scratch for the prefix partials. A caller that
+ * only ever receives its input and output buffers, such as an operator plugin inside an
+ * inference engine that owns the whole device heap and hands its plugins no allocator,
+ * has no way to provide it. This call instead uses a fixed 16 MiB array that lives in
+ * the library's own device memory (every GPU that loads the library holds it until the
+ * process exits) and allocates nothing. Arguments and results are those of
+ * ls_verify_attn.
+ *
+ *   - Returns LS_ERR_WORKSPACE if these dims need more than 16 MiB of scratch (see
+ *     ls_verify_attn_workspace_size); use ls_verify_attn with a workspace for those.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before capturing any stream.
+ *   - All calls on a device share the one array, which keeps whatever the last call
+ *     left in it. Calls whose kernels overlap on the GPU (different streams without an
+ *     ordering between them) race on it and give wrong results; order them.
+ *   - Device-detected errors (bad tree, length mismatch, timeout) are recorded in the
+ *     shared array and cannot be read back through ls_verify_attn_check; callers that
+ *     need them use ls_verify_attn.
+ */
+LS_API int ls_verify_attn_static(const void* q, const void* k_cache, const void* v_cache,
+                                 const void* k_tree, const void* v_tree,
+                                 const int32_t* tree_parent, const int32_t* cu_seqlens,
+                                 void* out, float* lse, const ls_verify_dims* dims, void* stream);
+
+/*
  * Waits for `stream`, then reads the device-side status that the last ls_verify_attn
  * call with this workspace and these dims recorded. Returns LS_OK, LS_ERR_BAD_TREE,
  * LS_ERR_LENGTHS, LS_ERR_TIMEOUT, or LS_ERR_CUDA if the copy itself failed.

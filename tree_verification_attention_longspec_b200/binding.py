@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3:
                 4: "LS_ERR_CUDA", 5: "LS_ERR_BAD_TREE", 6: "LS_ERR_TIMEOUT", 7: "LS_ERR_LENGTHS"}
 EXPORTED = ("ls_verify_attn", "ls_verify_attn_prefix", "ls_verify_attn_tree_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
-            "ls_verify_attn_plan")
+            "ls_verify_attn_plan", "ls_verify_attn_static")
 
 
 class LSError(RuntimeError):
@@ -63,6 +63,8 @@ def load_library(path: str = LIB_PATH):
     lib.ls_verify_attn_prefix.restype = ctypes.c_int
     lib.ls_verify_attn_tree_combine.argtypes = [P, P, P, P, P, P, P, D, P, ctypes.c_size_t, P]
     lib.ls_verify_attn_tree_combine.restype = ctypes.c_int
+    lib.ls_verify_attn_static.argtypes = [P, P, P, P, P, P, P, P, P, D, P]
+    lib.ls_verify_attn_static.restype = ctypes.c_int
     lib.ls_verify_attn_workspace_size.argtypes = [D]
     lib.ls_verify_attn_workspace_size.restype = ctypes.c_size_t
     lib.ls_verify_attn_check.argtypes = [D, P, P]
@@ -111,6 +113,14 @@ def call_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, out, lse, 
     return int(load_library().ls_verify_attn(q, k_cache, v_cache, k_tree, v_tree, parent,
                                              cu_seqlens, out, lse, ctypes.byref(dims), workspace,
                                              workspace_bytes, stream))
+
+
+def call_static_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, out, lse, dims: Dims,
+                    stream) -> int:
+    """ls_verify_attn_static on raw device addresses (ints): no workspace argument, for
+    callers that cannot allocate device memory; returns the status code."""
+    return int(load_library().ls_verify_attn_static(q, k_cache, v_cache, k_tree, v_tree, parent,
+                                                    cu_seqlens, out, lse, ctypes.byref(dims), stream))
 
 
 def call_prefix_raw(q, k_cache, v_cache, cu_seqlens, dims: Dims, workspace, workspace_bytes: int,
