@@ -74,6 +74,19 @@ def config_of(inp, l2_note):
             "total_prefix_len": int(L.sum()), "seed": inp.seed, "l2": l2_note}
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of `values` over all ranks (the step time of a multi-GPU run
+    is that of its slowest rank); the values themselves when running alone."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons of one GPU through NVML in a thread."""
@@ -313,10 +326,7 @@ def run_ours(args):
     prefix_ms = [e[0].elapsed_time(e[1]) for e in evp]
     ms_per_step = float(statistics.mean(step_ms))
     prefix_avg_ms = float(statistics.mean(prefix_ms))
-    if world > 1:
-        t = torch.tensor([ms_per_step, prefix_avg_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step, prefix_avg_ms = float(t[0]), float(t[1])
+    ms_per_step, prefix_avg_ms = max_over_ranks([ms_per_step, prefix_avg_ms], device=dev)
     st = op.check()
     if st != 0:
         raise binding.LSError(st, "device status after timing")
@@ -347,10 +357,7 @@ def run_ours(args):
             if k >= 2:
                 times.append(e0.elapsed_time(e1))
         e2e_ms = float(statistics.mean(times))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = max_over_ranks([e2e_ms], device=dev)[0]
         e2e = {"value": e2e_ms * 1000.0 / world, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": n_e2e}
 
