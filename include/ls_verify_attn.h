@@ -143,12 +143,12 @@ LS_API int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const 
  * ls_verify_attn needs caller-provided scratch for the prefix partials. A caller that
  * only ever receives its input and output buffers, such as an operator plugin inside an
  * inference engine that owns the whole device heap and hands its plugins no allocator,
- * has no way to provide it. This call instead uses a fixed 16 MiB array that lives in
+ * has no way to provide it. This call instead uses a fixed 32 MiB array that lives in
  * the library's own device memory (every GPU that loads the library holds it until the
  * process exits) and allocates nothing. Arguments and results are those of
  * ls_verify_attn.
  *
- *   - Returns LS_ERR_WORKSPACE if these dims need more than 16 MiB of scratch (see
+ *   - Returns LS_ERR_WORKSPACE if these dims need more than 32 MiB of scratch (see
  *     ls_verify_attn_workspace_size); use ls_verify_attn with a workspace for those.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before capturing any stream.

@@ -1,4 +1,4 @@
-// Host-side check of the chunk plan: every (sequence, kv head, row group, 128-key
+// Host-side check of the chunk plan: every (sequence, kv head, unit, 128-key
 // block) of the prefix is covered by exactly one chunk, chunk ids are dense, and the
 // per-sequence chunk ranges that the combine kernel uses agree with locate_chunk.
 // Usage: plan_check B Hq Hkv T C uniform_n L_0 ... L_{B-1}   (exit 0 = pass)
@@ -22,7 +22,8 @@ int main(int argc, char** argv) {
   p.d = 128;
   p.g = p.Hq / p.Hkv;
   p.rows = p.T * p.g;
-  p.rg = ls::ceil_div(p.rows, ls::kUnitRows);
+  p.tpu = ls::kUnitRows / p.g;
+  p.rg = ls::ceil_div(p.T, p.tpu);
   if (argc != 7 + p.B) return 2;
   std::vector<int32_t> cu(p.B + 1, 0);
   for (int b = 0; b < p.B; ++b) cu[b + 1] = cu[b] + atoi(argv[7 + b]);

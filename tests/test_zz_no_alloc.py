@@ -20,7 +20,7 @@ from tree_verification_attention_longspec_b200.inputs import Workload, make_inpu
 
 pytestmark = pytest.mark.gpu
 
-STATIC_SCRATCH_BYTES = 16 << 20
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def _static_call(dev, dims, out, lse):

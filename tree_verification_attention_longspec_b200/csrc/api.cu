@@ -77,7 +77,9 @@ int make_plan(const ls_verify_dims* d, Plan* p) {
   q.T = d->tree_size;
   q.g = q.Hq / q.Hkv;
   q.rows = q.T * q.g;
-  q.rg = ls::ceil_div(q.rows, ls::kUnitRows);
+  if (q.g > ls::kUnitRows) return LS_ERR_UNSUPPORTED;
+  q.tpu = ls::kUnitRows / q.g;
+  q.rg = ls::ceil_div(q.T, q.tpu);
   q.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)q.d);
   q.scale_log2 = (float)((double)q.scale * 1.4426950408889634074);
   q.n_combine = q.B * q.T * q.Hkv;

@@ -1,12 +1,13 @@
 // Work split and workspace layout shared by the host launcher and the kernels.
 //
 // The prefix ("Cached-Teil") work is cut into chunks. A chunk is one
-// (sequence b, kv head kh, row group rg, key range) and becomes one CTA of the
-// prefix kernel. A row group is 128 query rows of one kv head; the rows of a kv
-// head are its T*g (tree node, head-in-group) pairs, row r = i*g + j.
-// Every chunk of a sequence covers C consecutive 128-key blocks (the last one
-// fewer), so the chunk grid follows from the prefix lengths and C alone, and the
-// device recomputes it from cu_seqlens without any table in memory.
+// (sequence b, kv head kh, unit u, key range) and becomes one CTA of the prefix
+// kernel. The query rows of a kv head are its T*g (tree node i, head-in-group j)
+// pairs; a unit holds the rows of tpu = floor(256 / g) consecutive tree nodes, so its
+// rows are whole nodes (at most 256 of them, row (i - u*tpu)*g + j of the unit) and
+// one TMA box brings them in. Every chunk of a sequence covers C consecutive 128-key
+// blocks (the last one fewer), so the chunk grid follows from the prefix lengths and
+// C alone, and the device recomputes it from cu_seqlens without any table in memory.
 #pragma once
 #include <stdint.h>
 
@@ -19,7 +20,7 @@
 namespace ls {
 
 constexpr int kBlockN = 128;       // keys per block of the prefix loop
-constexpr int kUnitRows = 128;     // query rows per prefix chunk (one 128-row MMA tile)
+constexpr int kUnitRows = 256;     // query rows per prefix chunk (two 128-row MMA tiles)
 constexpr int kMaxTree = 128;      // largest supported tree
 
 // device-side status bits (combined into one LS_ERR_* by ls_verify_attn_check)
@@ -30,7 +31,8 @@ constexpr uint32_t kErrTimeout = 4u;
 struct Plan {
   int32_t B, Hq, Hkv, d, T, g;
   int32_t rows;        // T * g query rows per (sequence, kv head)
-  int32_t rg;          // row groups per (sequence, kv head): ceil(rows / 128)
+  int32_t tpu;         // tree nodes per unit: floor(kUnitRows / g)
+  int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
   int32_t C;           // 128-key blocks per chunk
   int32_t uniform_n;   // >= 0: chunks per unit for every sequence; -1: from L_b
   int32_t n_chunks;    // prefix CTAs
@@ -41,15 +43,21 @@ struct Plan {
 
 LS_HD int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
 
-// chunks of one (sequence, kv head, row group) unit for a prefix of L keys
+// chunks of one (sequence, kv head, unit) for a prefix of L keys
 LS_HD int32_t chunks_per_unit(const Plan& p, int32_t L) {
   if (p.uniform_n >= 0) return p.uniform_n;
   if (L <= 0) return 0;
   return ceil_div(ceil_div(L, kBlockN), p.C);
 }
 
+// Unit and row inside the unit of query row (tree node i, head-in-group j).
+LS_HD void unit_row(const Plan& p, int32_t i, int32_t j, int32_t* unit, int32_t* row) {
+  *unit = i / p.tpu;
+  *row = (i - *unit * p.tpu) * p.g + j;
+}
+
 struct ChunkCoord {
-  int32_t b, kh, rgi, split, n_split;  // sequence, kv head, row group, split index, splits of unit
+  int32_t b, kh, rgi, split, n_split;  // sequence, kv head, unit, split index, splits of unit
   int32_t key_begin, key_end;          // key range inside the sequence's prefix
   int32_t seq_offset;                  // cu_seqlens[b]
   bool valid;
@@ -104,8 +112,8 @@ LS_HD void sequence_chunks(const Plan& p, const int32_t* cu, int32_t b, int32_t*
 
 // Workspace layout (byte offsets, each 256-aligned).
 struct Layout {
-  uint64_t o_part;        // float [n_chunks][128][d]   prefix partial out, normalised
-  uint64_t lse_part;      // float [n_chunks][128]      prefix partial lse, log2 domain
+  uint64_t o_part;        // float [n_chunks][kUnitRows][d]   prefix partial out, normalised
+  uint64_t lse_part;      // float [n_chunks][kUnitRows]      prefix partial lse, log2 domain
   uint64_t chunk_status;  // u32   [n_chunks]
   uint64_t status;        // u32   [n_combine]
   uint64_t total;

@@ -20,7 +20,7 @@
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB
 constexpr int kMaxDevices = 64;
 
 // The scratch itself. Host code must not use its name as a pointer: on the host it is

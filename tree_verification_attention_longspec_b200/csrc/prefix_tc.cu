@@ -4,30 +4,29 @@
 // mask, and it carries most of the work, so it runs on the fastest path. With grouped-
 // query attention the T*g (tree node, head-in-group) rows of one kv head share every
 // key, so the prefix step is a dense contraction: S = Q K^T and O += P V. One CTA handles
-// one chunk: a 128-row tile of one (sequence, kv head) against a range of 128-key
-// blocks, and leaves its partial (out normalised by its own sum, lse in the log2
-// domain) for the combine kernel.
+// one chunk: a 256-row unit of one (sequence, kv head), as two 128-row query tiles,
+// against a range of 128-key blocks, and leaves its partial (out normalised by its own
+// sum, lse in the log2 domain) for the combine kernel.
 //
-// Pipeline. The scores of key block j go to one of two 128-column TMEM buffers (j % 2),
-// so the tensor core computes S(j+1) = Q K(j+1)^T while the softmax works on S(j).
-// The two softmax warpgroups split every block's columns: warpgroup x owns keys
-// [64x, 64x+64) of each block and keeps its own running max m_x, sum l_x and output
-// accumulator O_x += P_x V_x in TMEM, so the halves never wait for each other; they are
-// merged by log-sum-exp once, at the end. P_x (bf16) is written over the scores it came
-// from and read by the PV product straight from TMEM.
+// Ping-pong. Each query tile t has one softmax warpgroup, one score buffer S_t and one
+// output accumulator O_t in TMEM. The MMA thread walks the key blocks and, per block j,
+// issues O_0 += P_0(j) V(j), S_0(j+1) = Q_0 K(j+1)^T, then the same for tile 1. While
+// the tensor core works for one tile, the other tile's warpgroup runs its softmax, so
+// the exponentials of one tile overlap the other tile's MMAs, and the special-function
+// unit (MUFU), which bounds the softmax, is shared by two warpgroups that are out of
+// phase. Every K/V tile staged in shared memory serves both query tiles.
 //
 // Warp roles (320 threads, one CTA per SM):
-//   warps 0-3  softmax of key half 0, warps 4-7 of key half 1: one thread per query
-//              row (= TMEM lane). P is computed against the current m_x in one pass;
-//              only when a block's maximum exceeds m_x by more than 2^8 is m_x raised,
-//              O_x rescaled in TMEM and P recomputed.
+//   warps 0-3  softmax of tile 0, warps 4-7 of tile 1: one thread per query row (= TMEM
+//              lane) holding the block's 128 scores. P is computed against the running
+//              max m in one pass; only when a block's maximum exceeds m by more than 2^8
+//              is m raised and O_t rescaled in TMEM. P (bf16) overwrites the scores in
+//              two halves of 64 keys, each announced on its own barrier, so the MMA
+//              thread starts on the first half while the second is computed.
 //   warp 8     TMA producer: streams 128-key K and V blocks into a ring of slots.
 //   warp 9     MMA issuer (one thread): S = Q K^T (shared-memory operands, N = 128) and
-//              O_x += P_x V_x (P from TMEM, K = 64, N = d), tcgen05.commit to mbarriers.
-//              It waits once per block and then issues the block's 16 MMAs back to back:
-//              MMA issue is throttled to the tensor pipe's pace, so every pause of this
-//              thread is idle tensor time.
-// TMEM columns (512 allocated): score buffer u at 128u, O_x at 256 + d*x.
+//              O += P V (P from TMEM, N = d), tcgen05.commit to mbarriers.
+// TMEM columns (512 allocated): S_t at 128 t, O_t at 256 + d t.
 // Every wait is bounded: on a timeout the CTA raises an abort flag, all roles drain
 // their in-flight copies and MMAs, TMEM is freed, and the chunk status reports it.
 #include <cudaTypedefs.h>
@@ -45,44 +44,70 @@ constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kMaxSlots = 12;
-constexpr int kHalf = 64;  // keys of a block owned by one softmax warpgroup
+constexpr int kTiles = 2;  // 128-row query tiles per CTA
+constexpr int kHalf = 64;  // keys per P half
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+static_assert(kUnitRows == kTiles * 128, "a unit is two 128-row tiles");
 
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;             // 128 rows x 64 bf16, 128B-swizzled
   static constexpr int kTileBytes = kPanels * kPanelBytes;  // 128 rows x D bf16
-  static constexpr int kSlots = D == 128 ? 6 : 12;
+  static constexpr int kSlots = D == 128 ? 5 : 12;
+  // Q: [panel][kUnitRows rows][128 B]; tile t is rows [128 t, 128 t + 128) of each panel
+  static constexpr int kQPanelBytes = kUnitRows * 128;
   static constexpr int kQOff = 0;
-  static constexpr int kSlotOff = kTileBytes;
+  static constexpr int kSlotOff = kPanels * kQPanelBytes;
   static constexpr int kBarOff = kSlotOff + kSlots * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 1024 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColO = 256;
+  static constexpr uint32_t kColS = 0;    // S_t / P_t at 128 t
+  static constexpr uint32_t kColO = 256;  // O_t at 256 + D t
   static_assert(kSlots <= kMaxSlots, "slots");
-  static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(kPanels * kQPanelBytes >= 128 * D * 4 && kSlots * kTileBytes >= 128 * D * 4, "epilogue staging");
 };
 
 struct alignas(64) TcParams {
+  CUtensorMap tmap_q;
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   PrefixArgs a;
 };
 
 struct Bars {
+  uint64_t q_full;  // the unit's Q rows are in shared memory
   uint64_t full[kMaxSlots];
   uint64_t empty[kMaxSlots];
-  uint64_t s_full[2];     // [buffer]: S(j) of buffer j%2 is in TMEM
-  uint64_t p_full[2][2];  // [half][buffer]: P_x(j) is in TMEM
-  uint64_t pv_last;       // O += P(nb-2) V(nb-2) finished (lets the last block rescale O)
-  uint64_t o_full;
+  uint64_t s_full[kTiles];     // S_t(j) is in TMEM (and O_t holds every PV before it)
+  uint64_t p_full[kTiles][2];  // half h of P_t(j) is in TMEM
+  uint64_t o_full[kTiles];     // every MMA of tile t finished
   uint32_t tmem_base;
   uint32_t abort;
 };
-static_assert(sizeof(Bars) <= 1024, "barrier block");
+
+// The kernel asks for the whole dynamic window a CTA may have and aligns its layout up
+// to 1024 bytes inside it (the 128-byte swizzle atom repeats every 1024 bytes).
+constexpr int kSmemWindow = 232448;
+template <int D>
+constexpr int smem_need() {
+  return Cfg<D>::kBarOff + (int)sizeof(Bars) + 1024;
+}
+static_assert(smem_need<128>() <= kSmemWindow && smem_need<64>() <= kSmemWindow, "shared memory");
+
+// AND of `pred` over the `n` threads that meet at named barrier `id`.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 
 // Waits only on time (used to drain in-flight work after an abort).
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -90,8 +115,8 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return mbar_wait_bounded(bar, parity, &never, kTimeoutNs);
 }
 
-// P = 2^(s*cs - m) for the 64 scores this thread holds, packed to bf16 pairs; adds the
-// values to (sum0, sum1). EMU of every 4 pairs use the FMA-pipe exponential.
+// P = 2^(s*cs - m) for 64 scores, packed to bf16 pairs; adds the values to (sum0, sum1).
+// EMU of every 4 pairs use the FMA-pipe exponential.
 template <int EMU>
 __device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float m, uint32_t (&pk)[kHalf / 2],
                                        float& sum0, float& sum1) {
@@ -114,8 +139,8 @@ __device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float 
 template <int D, int EMU>
 __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_constant__ TcParams P) {
   using C = Cfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
   const PrefixArgs& a = P.a;
   const Plan& p = a.p;
@@ -126,27 +151,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
   const int n_keys = c.key_end - c.key_begin;
   const int nb = (n_keys + kBlockN - 1) / kBlockN;
   const int tail_shift = nb * kBlockN - n_keys;  // masked leading columns of the last block
-  const int row0 = c.rgi * kUnitRows;
-  const int rows_here = min(kUnitRows, p.rows - row0);
-
+  const int tok0 = c.rgi * p.tpu;                    // first tree node of the unit
+  const int rows_here = min(p.tpu, p.T - tok0) * p.g;  // rows of the unit that exist
   if (nb == 0) {  // empty key range: an empty partial
-    if (tid < rows_here) a.lse_part[(size_t)blockIdx.x * kUnitRows + tid] = -INFINITY;
+    for (int r = tid; r < rows_here; r += kThreads) a.lse_part[(size_t)blockIdx.x * kUnitRows + r] = -INFINITY;
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
     return;
   }
 
   if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(&bars->s_full[u], 1);
-      mbar_init(&bars->p_full[0][u], 128);
-      mbar_init(&bars->p_full[1][u], 128);
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t][0], 128);
+      mbar_init(&bars->p_full[t][1], 128);
     }
-    mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->pv_last, 1);
+    mbar_init(&bars->o_full[0], 1);
+    mbar_init(&bars->o_full[1], 1);
     bars->abort = 0u;
     fence_mbar_init();
   }
@@ -155,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
     tmem_relinquish();
   }
   if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_map(&P.tmap_q);
     tma_prefetch_map(&P.tmap_k);
     tma_prefetch_map(&P.tmap_v);
   }
@@ -169,15 +195,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
+    // Ring order = consumption order: K(0), V(0), K(1), V(1), ...
     if (lane == 0) {
-      int issued = 0;
-      for (int j = 0; j < nb; ++j) {
+      // Q first: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows
+      // past the batch's last node read as zeros)
+      mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn)
+        tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
+                    c.b * p.T + tok0);
+      int issued = 0, slot = 0, use = 0;
+      bool ok = true;
+      for (int j = 0; j < nb && ok; ++j) {
         int key0 = c.key_begin + j * kBlockN;
         if (j == nb - 1) key0 -= tail_shift;  // the box ends at the sequence end
-        const int grow = c.seq_offset + key0;
-        bool ok = true;
         for (int kv = 0; kv < 2; ++kv) {
-          const int seq = 2 * j + kv, slot = seq % C::kSlots, use = seq / C::kSlots;
           if (!mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs)) {
             ok = false;
             break;
@@ -187,38 +219,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
           const CUtensorMap* map = kv ? &P.tmap_v : &P.tmap_k;
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, grow);
+            tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, c.seq_offset + key0);
           ++issued;
+          if (++slot == C::kSlots) {
+            slot = 0;
+            ++use;
+          }
+          // K(0) alone first: at start-up every CTA asks for just Q and one tile, so those
+          // arrive quickly instead of sharing the memory system with the whole ring's fill
+          if (issued == 1 && !mbar_wait_bounded(&bars->full[0], 0, abort, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
         }
-        if (!ok) break;
       }
       // make sure no copy is still writing shared memory when the CTA ends
+      drain_wait(&bars->q_full, 0);
       const int first = issued > C::kSlots ? issued - C::kSlots : 0;
       for (int seq = first; seq < issued; ++seq)
         drain_wait(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ load Q (warps 0-7)
+    // ------------------------------------------------------------------ Q padding (warps 0-7)
+    // The TMA box fills rows [0, tpu*g) of each Q panel; the (fewer than g) rows after
+    // it are zeroed here so that no stale shared memory enters an MMA.
     if (warp < 8) {
-      const int chunks_per_row = D / 8;  // 16-byte chunks
-      const int total = 128 * chunks_per_row;
-      for (int idx = tid; idx < total; idx += 256) {
-        const int r = idx / chunks_per_row, ch = idx % chunks_per_row;
-        const int rg = row0 + r;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (rg < p.rows) {
-          const int i = rg / p.g, jh = rg % p.g;
-          const uint16_t* src = a.q + ((size_t)(c.b * p.T + i) * p.Hq + c.kh * p.g + jh) * D + ch * 8;
-          v = *reinterpret_cast<const uint4*>(src);
-        }
-        const int pn = ch >> 3, cc = ch & 7;
-        uint8_t* dst = smem + C::kQOff + pn * C::kPanelBytes + r * 128 + ((cc ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = v;
+      const int pad0 = p.tpu * p.g;
+      const int n16 = (kUnitRows - pad0) * 8;  // 16-byte chunks per panel
+      for (int idx = tid; idx < C::kPanels * n16; idx += 256) {
+        const int pn = idx / n16, k = idx % n16;
+        *reinterpret_cast<uint4*>(smem + C::kQOff + pn * C::kQPanelBytes + pad0 * 128 + k * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
     }
-    // Q is in shared memory: warps 0-7 and the MMA warp meet at named barrier 1
+    // the padding is in shared memory: warps 0-7 and the MMA warp meet at barrier 1
     if (warp < 8 || warp == kMmaWarp) asm volatile("bar.sync 1, 288;" ::: "memory");
 
     if (warp == kMmaWarp) {
@@ -229,220 +265,242 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
         // A descriptor differs from another of the same kind only in its start-address
         // field (address >> 4 in the low 14 bits; shared addresses stay below 256 KB, so
         // adding an offset never carries out of it): build the bases once, add offsets.
-        const uint64_t dq = umma_sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+        const uint64_t dq0 = umma_sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+        constexpr uint32_t kQPanel16 = C::kQPanelBytes >> 4, kQTile16 = (128 * 128) >> 4;
         const uint64_t dk0 = umma_sdesc_sw128(smem_u32(smem + C::kSlotOff), 16, 1024);
         const uint64_t dv0 = umma_sdesc_sw128(smem_u32(smem + C::kSlotOff), C::kPanelBytes, 1024);
         constexpr uint32_t kTile16 = C::kTileBytes >> 4, kPanel16 = C::kPanelBytes >> 4;
-        // K block j is sequence 2j of the slot ring, V block j is sequence 2j+1
-        auto wait_full = [&](int seq) {
-          return mbar_wait_bounded(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1, abort, kTimeoutNs);
-        };
-        // S(j) = Q K(j)^T into score buffer j%2; K(j) sits in ring slot `slot`
-        auto issue_qk = [&](int j, int slot) {
+        // S_t = Q_t K^T into tile t's score buffer; K sits in ring slot `slot`
+        auto issue_qk = [&](int t, int slot) {
+          const uint64_t dq = dq0 + (uint64_t)(t * kQTile16);
           const uint64_t dk = dk0 + (uint64_t)(slot * kTile16);
-          const uint32_t tS = tbase + C::kColS + (j & 1) * kBlockN;
+          const uint32_t tS = tbase + C::kColS + t * kBlockN;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPanel16 + (kk & 3) * 2;  // 16-byte units
-            umma_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+            const uint32_t koff = (kk & 3) * 2;  // 32 bytes per K step inside a panel (16-byte units)
+            umma_ss(tS, dq + (kk >> 2) * kQPanel16 + koff, dk + (kk >> 2) * kPanel16 + koff, idesc_qk,
+                    kk > 0 ? 1u : 0u);
           }
-          umma_commit(&bars->s_full[j & 1]);
+          umma_commit(&bars->s_full[t]);
         };
-        // O_x += P_x(j) V_x(j): K = 64 keys of half x, P from TMEM, V rows of that half;
-        // V(j) sits in ring slot `slot`
-        auto issue_pv = [&](int x, int j, int slot) {
-          const uint64_t dv = dv0 + (uint64_t)(slot * kTile16 + x * (kHalf * 128 / 16));
-          const uint32_t tP = tbase + C::kColS + (j & 1) * kBlockN + x * kHalf;
-          const uint32_t tO = tbase + C::kColO + x * D;
+        // O_t += P_t V over keys [64h, 64h+64) of block j: four K = 16 steps, P from TMEM
+        auto issue_pv = [&](int t, int slot, int j, int h) {
+          const uint64_t dv = dv0 + (uint64_t)(slot * kTile16);
+          const uint32_t tP = tbase + C::kColS + t * kBlockN;
+          const uint32_t tO = tbase + C::kColO + t * D;
 #pragma unroll
-          for (int kk = 0; kk < kHalf / 16; ++kk)
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;
             umma_ts(tO, tP + kk * 8, dv + kk * (2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
         };
-        bool ok = wait_full(0);
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+          const bool got = mbar_wait_bounded(bar, parity, abort, kTimeoutNs);
+          if (got) tc_fence_after_sync();
+          return got;
+        };
+        int slot = 0, use = 0;  // ring position of the next tile, in consumption order
+        auto advance = [&]() {
+          if (++slot == C::kSlots) {
+            slot = 0;
+            use ^= 1;
+          }
+        };
+        bool ok = wait(&bars->q_full, 0) && wait(&bars->full[slot], use);  // Q, K(0)
         if (ok) {
-          tc_fence_after_sync();
-          issue_qk(0, 0);
-          umma_commit(&bars->empty[0]);
-          if (nb > 1) {
-            ok = wait_full(2);
-            if (ok) {
-              tc_fence_after_sync();
-              issue_qk(1, 2 % C::kSlots);
-              umma_commit(&bars->empty[2 % C::kSlots]);
+          issue_qk(0, slot);
+          issue_qk(1, slot);
+          umma_commit(&bars->empty[slot]);
+          advance();
+        }
+        for (int j = 0; j < nb && ok; ++j) {
+          const int sv = slot, uv = use;  // V(j)
+          advance();
+          const bool more = j + 1 < nb;
+          const int sk = slot, uk = use;  // K(j+1), when there is one
+          const uint32_t pp = j & 1;
+          ok = wait(&bars->full[sv], uv);
+          for (int t = 0; t < kTiles && ok; ++t) {
+            ok = wait(&bars->p_full[t][0], pp);
+            if (!ok) break;
+            issue_pv(t, sv, j, 0);
+            ok = wait(&bars->p_full[t][1], pp);
+            if (!ok) break;
+            issue_pv(t, sv, j, 1);
+            if (!more && t == 0) umma_commit(&bars->o_full[0]);  // tile 0's epilogue may start
+            if (more) {
+              if (t == 0) ok = wait(&bars->full[sk], uk);
+              if (!ok) break;
+              issue_qk(t, sk);
             }
           }
-        }
-        // One wait point per block, then all of the block's MMAs back to back:
-        // O_x += P_x(j) V_x(j) for both halves, then S(j+2) into buffer j%2 (whose P(j)
-        // has just been consumed). Three commits per block: V(j)'s slot, S(j+2) and
-        // K(j+2)'s slot. Slot indices and phases advance incrementally (V(j) is sequence
-        // 2j+1, K(j+2) is sequence 2j+4 of the ring).
-        int sv = 1 % C::kSlots, uv = 1 / C::kSlots;  // V(j): slot and use count parity
-        int sk = 4 % C::kSlots, uk = 4 / C::kSlots;  // K(j+2)
-        for (int j = 0; j < nb && ok; ++j) {
-          const bool more = j + 2 < nb;
-          uint64_t* bk = more ? &bars->full[sk] : &bars->full[sv];  // no K(j+2): test V twice
-          const uint32_t pk = more ? (uk & 1) : (uv & 1);
-          const uint32_t pp = (j >> 1) & 1;
-          if (!mbar_try_wait4(&bars->full[sv], uv & 1, bk, pk, &bars->p_full[0][j & 1], pp,
-                              &bars->p_full[1][j & 1], pp)) {
-            ok = mbar_wait_bounded(&bars->full[sv], uv & 1, abort, kTimeoutNs) &&
-                 mbar_wait_bounded(bk, pk, abort, kTimeoutNs) &&
-                 mbar_wait_bounded(&bars->p_full[0][j & 1], pp, abort, kTimeoutNs) &&
-                 mbar_wait_bounded(&bars->p_full[1][j & 1], pp, abort, kTimeoutNs);
-            if (!ok) break;
-          }
-          tc_fence_after_sync();
-          issue_pv(0, j, sv);
-          issue_pv(1, j, sv);
+          if (!ok) break;
           umma_commit(&bars->empty[sv]);
-          if (j == nb - 2) umma_commit(&bars->pv_last);
           if (more) {
-            issue_qk(j + 2, sk);
             umma_commit(&bars->empty[sk]);
+            advance();
           }
-          sv += 2;
-          if (sv >= C::kSlots) { sv -= C::kSlots; uv ^= 1; }
-          sk += 2;
-          if (sk >= C::kSlots) { sk -= C::kSlots; uk ^= 1; }
         }
-        umma_commit(&bars->o_full);
-        drain_wait(&bars->o_full, 0);
+        // tile 0's last PV precedes tile 1's in issue order, so o_full[1] completes last
+        umma_commit(&bars->o_full[1]);
+        drain_wait(&bars->o_full[1], 0);
       }
       __syncwarp();
     } else {
       // ---------------------------------------------------------------- softmax / epilogue
-      const int x = warp >> 2;  // key half
-      const int row = (warp & 3) * 32 + lane;
+      const int t = warp >> 2;                 // query tile
+      const int row = (warp & 3) * 32 + lane;  // row of the tile = TMEM lane
       const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-      const uint32_t tS0 = tbase + lane_base + C::kColS + x * kHalf;
-      const uint32_t tOx = tbase + lane_base + C::kColO + x * D;
+      const uint32_t tS = tbase + lane_base + C::kColS + t * kBlockN;
+      const uint32_t tO = tbase + lane_base + C::kColO + t * D;
       const float cs = p.scale_log2;
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
       bool ok = true;
       for (int j = 0; j < nb; ++j) {
-        const int u = j & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[u], (j >> 1) & 1, abort, kTimeoutNs));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], j & 1, abort, kTimeoutNs));
         if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t tS = tS0 + u * kBlockN;
-        float s[kHalf];
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tS, r0);
-          tmem_ld32(tS + 32, r1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            s[e] = __uint_as_float(r0[e]);
-            s[32 + e] = __uint_as_float(r1[e]);
-          }
-        }
-        // the sequence's last block: columns before tail_shift belong to earlier keys
-        const int shift = j == nb - 1 ? tail_shift - x * kHalf : 0;
-        if (shift > 0) {
-#pragma unroll
-          for (int e = 0; e < kHalf; ++e)
-            if (e < shift) s[e] = -INFINITY;
-        }
+        // All 128 scores for the row maximum; the scores of keys 0..63 stay in registers
+        // for P's first half, those of keys 64..127 are read again for the second half.
+        float lo[kHalf];
         float mx;
+        const int shift = j == nb - 1 ? tail_shift : 0;  // masked leading columns
         {
-          float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+          uint32_t r[4][32];
 #pragma unroll
-          for (int e = 4; e < kHalf; e += 8) {
-            m0 = fmax3(m0, s[e], s[e + 1]);
-            m1 = fmax3(m1, s[e + 2], s[e + 3]);
-            m2 = fmax3(m2, s[e + 4], s[e + 5]);
-            m3 = fmax3(m3, s[e + 6], s[e + 7]);
+          for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, r[q]);
+          tmem_wait_ld();
+          float hi[kHalf];
+#pragma unroll
+          for (int e = 0; e < kHalf; ++e) {
+            lo[e] = __uint_as_float(r[e >> 5][e & 31]);
+            hi[e] = __uint_as_float(r[2 + (e >> 5)][e & 31]);
           }
-          mx = fmax3(m0, m1, fmaxf(m2, m3)) * cs;  // -inf if the whole half is masked
+          if (shift > 0) {  // the sequence's last block: these columns are earlier keys
+#pragma unroll
+            for (int e = 0; e < kHalf; ++e) {
+              if (e < shift) lo[e] = -INFINITY;
+              if (e + kHalf < shift) hi[e] = -INFINITY;
+            }
+          }
+          float m0 = fmaxf(lo[0], hi[0]), m1 = fmaxf(lo[1], hi[1]);
+          float m2 = fmaxf(lo[2], hi[2]), m3 = fmaxf(lo[3], hi[3]);
+#pragma unroll
+          for (int e = 4; e < kHalf; e += 4) {
+            m0 = fmax3(m0, lo[e], hi[e]);
+            m1 = fmax3(m1, lo[e + 1], hi[e + 1]);
+            m2 = fmax3(m2, lo[e + 2], hi[e + 2]);
+            m3 = fmax3(m3, lo[e + 3], hi[e + 3]);
+          }
+          mx = fmax3(m0, m1, fmaxf(m2, m3)) * cs;
         }
-        uint32_t pk[kHalf / 2];
-        float sum0 = 0.f, sum1 = 0.f;
         const bool raise = mx > m + kRescaleThreshold;
-        if (__any_sync(0xffffffffu, raise)) {
-          // the maximum moved up: rescale what O_x and l hold (once the previous PV has
-          // landed) and compute P against the new maximum
-          const float m_new = raise ? mx : m;
-          if (j > 0) {
-            // O_x must hold all of PV(j-1) before it is rescaled. QK(j+1) was issued after
-            // PV(j-1), so S(j+1) being ready implies it; the last block has no S(j+1) and
-            // waits for the commit issued after PV(nb-2) instead.
-            ok = __all_sync(0xffffffffu, j + 1 < nb ? mbar_wait_bounded(&bars->s_full[(j + 1) & 1], ((j + 1) >> 1) & 1,
-                                                                        abort, kTimeoutNs)
-                                                    : mbar_wait_bounded(&bars->pv_last, 0, abort, kTimeoutNs));
-            if (!ok) break;
-            tc_fence_after_sync();
-            // f = 1 where m is unchanged; 0 where nothing was accumulated yet (m = -inf)
+        const bool any_raise = __any_sync(0xffffffffu, raise);
+        // masked columns (-inf) and the rare blocks that raise m take the MUFU-only path
+        const bool mufu_only = EMU == 0 || shift > 0 || any_raise;
+        const float m_new = raise ? mx : m;
+        float sum0 = 0.f, sum1 = 0.f;
+        {
+          uint32_t pk[kHalf / 2];
+          if (mufu_only) make_p<0>(lo, cs, m_new, pk, sum0, sum1);
+          else make_p<EMU>(lo, cs, m_new, pk, sum0, sum1);
+          if (any_raise) {
+            // the maximum moved up: rescale what O_t and l hold. O_t is idle: every PV of
+            // this tile issued before S_t(j) has completed (s_full), and PV_t(j) waits for
+            // this warpgroup's P. f = 1 where m is unchanged, 0 before the first block.
             const float f = m == m_new ? 1.f : ex2_approx(m - m_new);
+            if (j > 0) {
 #pragma unroll
-            for (int q4 = 0; q4 < D / 32; ++q4) {
-              uint32_t r[32];
-              tmem_ld32(tOx + q4 * 32, r);
-              tmem_wait_ld();
+              for (int q = 0; q < D / 16; ++q) {
+                uint32_t o[16];
+                tmem_ld16(tO + 16 * q, o);
+                tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-              tmem_st32(tOx + q4 * 32, r);
+                for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                tmem_st16(tO + 16 * q, o);
+              }
             }
             l *= f;
+            m = m_new;
           }
-          m = m_new;
+          tmem_st32(tS, pk);  // P over keys 0..63 -> columns 0..31
         }
-        // masked columns (-inf) and the rare blocks above take the MUFU-only path; while
-        // nothing has been seen yet (m = -inf, everything so far masked) every P is 0
-        if (EMU == 0 || shift > 0 || m == -INFINITY || __any_sync(0xffffffffu, raise)) {
-          make_p<0>(s, cs, m == -INFINITY ? 0.f : m, pk, sum0, sum1);
-        } else {
-          make_p<EMU>(s, cs, m, pk, sum0, sum1);
+        float hi[kHalf];
+        {
+          uint32_t r[2][32];
+          tmem_ld32(tS + 64, r[0]);  // P occupies columns 0..63 only: keys 64..127 are intact
+          tmem_ld32(tS + 96, r[1]);
+          tmem_wait_st();
+          tc_fence_before_sync();
+          mbar_arrive(&bars->p_full[t][0]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < kHalf; ++e) hi[e] = __uint_as_float(r[e >> 5][e & 31]);
+          if (shift > kHalf) {
+#pragma unroll
+            for (int e = 0; e < kHalf; ++e)
+              if (e + kHalf < shift) hi[e] = -INFINITY;
+          }
+        }
+        {
+          uint32_t pk[kHalf / 2];
+          if (mufu_only) make_p<0>(hi, cs, m, pk, sum0, sum1);
+          else make_p<EMU>(hi, cs, m, pk, sum0, sum1);
+          tmem_st32(tS + 32, pk);  // keys 64..127 -> columns 32..63
+          tmem_wait_st();
+          tc_fence_before_sync();
+          mbar_arrive(&bars->p_full[t][1]);
         }
         l += sum0 + sum1;
-        tmem_st32(tS, pk);
-        tmem_wait_st();
-        tc_fence_before_sync();
-        mbar_arrive(&bars->p_full[x][u]);
       }
       // -------------------------------------------------------------- epilogue
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full, 0, abort, kTimeoutNs));
-      // every MMA has finished (o_full), so the Q tile's shared memory is free: it carries
-      // both halves' (m, l) of every row to the other warpgroup
-      float* xm = reinterpret_cast<float*>(smem + C::kQOff);  // [2][128]
-      float* xl = xm + 256;                                   // [2][128]
-      xm[x * 128 + row] = ok ? m : -INFINITY;
-      xl[x * 128 + row] = ok ? l : 0.f;
-      asm volatile("bar.sync 2, 256;" ::: "memory");
-      if (ok) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full[t], 0, abort, kTimeoutNs));
+      // Each warpgroup stages its normalised 128 x D tile in shared memory (16-byte chunk
+      // c of row r at chunk c ^ (r & 7), conflict-free for the per-row writes) and then
+      // writes it out row-contiguously, since the tile's rows are contiguous in o_part.
+      // Tile 0 finishes while tile 1's last PV may still read V from the slot ring, so
+      // it stages over the Q tiles (every QK has completed by o_full[0]); tile 1, last of
+      // all, stages over the ring.
+      const bool ok_all = bar_and(2 + t, 128, ok);
+      if (ok_all) {
         tc_fence_after_sync();
-        const float ma = xm[row], mb = xm[128 + row];
-        const float M = fmaxf(ma, mb);
-        const float wa = ma == -INFINITY ? 0.f : ex2_approx(ma - M);
-        const float wb = mb == -INFINITY ? 0.f : ex2_approx(mb - M);
-        const float Ls = wa * xl[row] + wb * xl[128 + row];
-        const float inv = 1.f / Ls;
-        const float ca = wa * inv, cb = wb * inv;
-        const bool valid = row < rows_here;
-        // this warpgroup writes output columns [x*D/2, (x+1)*D/2) of its rows
-        float* dst = a.o_part + ((size_t)blockIdx.x * kUnitRows + row) * D + x * (D / 2);
-        const uint32_t tOa = tbase + lane_base + C::kColO + x * (D / 2);
-        const uint32_t tOb = tOa + D;
+        constexpr int kChunks = D / 4;  // float4 chunks per row
+        float* stage = reinterpret_cast<float*>(smem + (t == 0 ? C::kQOff : C::kSlotOff));
+        const float inv = 1.f / l;
 #pragma unroll
-        for (int q4 = 0; q4 < D / 64; ++q4) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tOa + q4 * 32, ra);
-          tmem_ld32(tOb + q4 * 32, rb);
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tO + 32 * q, r);
           tmem_wait_ld();
-          if (valid) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              float4 v;
-              v.x = fmaf(ca, __uint_as_float(ra[e]), cb * __uint_as_float(rb[e]));
-              v.y = fmaf(ca, __uint_as_float(ra[e + 1]), cb * __uint_as_float(rb[e + 1]));
-              v.z = fmaf(ca, __uint_as_float(ra[e + 2]), cb * __uint_as_float(rb[e + 2]));
-              v.w = fmaf(ca, __uint_as_float(ra[e + 3]), cb * __uint_as_float(rb[e + 3]));
-              *reinterpret_cast<float4*>(dst + q4 * 32 + e) = v;
-            }
+          for (int e = 0; e < 8; ++e) {
+            const int ch = 8 * q + e;
+            *reinterpret_cast<float4*>(stage + row * D + ((ch ^ (row & 7)) << 2)) =
+                make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                            __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
           }
         }
-        if (valid && x == 0) a.lse_part[(size_t)blockIdx.x * kUnitRows + row] = M + log2f(Ls);
+        const int ur = t * 128 + row;  // row of the unit
+        if (ur < rows_here) a.lse_part[(size_t)blockIdx.x * kUnitRows + ur] = m + log2f(l);
+        asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
+        const int tile_rows = min(128, max(0, rows_here - t * 128));
+        float* dst = a.o_part + ((size_t)blockIdx.x * kUnitRows + t * 128) * D;
+        const int wt = tid & 127;
+        const int n4 = tile_rows * kChunks;
+        for (int i0 = 0; i0 < n4; i0 += 8 * 128) {
+          float4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 128 + wt;
+            const int rr = i / kChunks, ch = i % kChunks;
+            if (i < n4) v[u] = *reinterpret_cast<const float4*>(stage + rr * D + ((ch ^ (rr & 7)) << 2));
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 128 + wt;
+            if (i < n4) *reinterpret_cast<float4*>(dst + (size_t)i * 4) = v[u];
+          }
+        }
       }
     }
   }
@@ -482,14 +540,29 @@ bool make_kv_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t row
   return r == CUDA_SUCCESS;
 }
 
+// Q viewed as [B*T nodes][H_kv][g][D] bf16; a box is 64 elements x g heads x one kv
+// head x tpu nodes, which lands as tpu*g consecutive 128-byte rows, node-major.
+bool make_q_map(CUtensorMap* map, const void* base, int D, const Plan& p) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)p.g, (cuuint64_t)p.Hkv, (cuuint64_t)p.B * p.T};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)p.g * D * 2, (cuuint64_t)p.Hq * D * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)p.g, 1, (cuuint32_t)p.tpu};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int EMU>
 cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) {
   TcParams P;
   P.a = a;
-  if (!make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows) ||
+  if (!make_q_map(&P.tmap_q, a.q, D, a.p) || !make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows) ||
       !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows))
     return cudaErrorInvalidValue;
-  const int smem = Cfg<D>::kSmemBytes;
+  const int smem = kSmemWindow;
   // opt in to the large shared-memory carve-out once per device
   static bool configured[64] = {};  // per template instance
   int dev = 0;

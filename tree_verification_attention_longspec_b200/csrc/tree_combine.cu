@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(256) tree_combine_kernel(CombineArgs a) {
   uint32_t err_w = 0;
   for (int j = warp; j < p.g; j += nwarps) {
     const size_t row = (size_t)tok * p.Hq + kh * p.g + j;
-    const int r = i * p.g + j;
-    const int rgi = r / kUnitRows, rl = r % kUnitRows;
+    int32_t rgi, rl;
+    unit_row(p, i, j, &rgi, &rl);
     const int cbase = chunk_first + (kh * p.rg + rgi) * chunk_per_unit;
     const int n_chunks = use_prefix ? chunk_per_unit : 0;
 
