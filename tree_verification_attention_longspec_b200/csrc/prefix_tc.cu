@@ -31,8 +31,6 @@
 // their in-flight copies and MMAs, TMEM is freed, and the chunk status reports it.
 #include <cudaTypedefs.h>
 
-#include <cstdlib>
-
 #include "ls_device.cuh"
 #include "sm100.cuh"
 
@@ -580,14 +578,12 @@ cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) 
 
 cudaError_t launch_prefix_tc(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) {
   if (a.p.n_chunks == 0) return cudaSuccess;
-  const char* env = getenv("LS_EMU");
-  const int emu = env ? atoi(env) : 0;
-  if (a.p.d == 64) return launch_d<64, 0>(a, kv_rows, stream);
-  switch (emu) {
-    case 1: return launch_d<128, 1>(a, kv_rows, stream);
-    case 2: return launch_d<128, 2>(a, kv_rows, stream);
-    default: return launch_d<128, 0>(a, kv_rows, stream);
-  }
+  // One pair of scores in four takes the FMA-pipe exponential: a quarter of the
+  // softmax's exponentials move off the special-function unit (MUFU), which is as busy
+  // as the tensor pipe at d = 128 and busier at d = 64. More than a quarter makes the
+  // FMA pipe the slower one.
+  if (a.p.d == 64) return launch_d<64, 1>(a, kv_rows, stream);
+  return launch_d<128, 1>(a, kv_rows, stream);
 }
 
 }  // namespace ls
