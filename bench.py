@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of tree-verification attention (LongSpec hybrid tree attention) on B200.
 
-One step = one full verification-attention call (prefix partials + tree/combine) over one
+One step = one full verification-attention call (partials kernel + combine kernel) over one
 batch of synthetic input of the named workload, inputs resident in HBM. L2 is flushed
 (a write of twice the L2 size) before every timed step, outside the timed events.
 
@@ -55,14 +55,15 @@ def workload_figures(inp):
     step_bytes = algorithmic_bytes(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.tree_size,
                                    total_L)
     step_flops = algorithmic_flops(w.num_q_heads, w.head_dim, w.tree_size, L)
-    # the prefix kernel alone: every (query row, prefix key) pair costs 4*d flops, and the
-    # prefix K/V plus the queries are its compulsory bytes
+    # the partials kernel (the dominant one) does every flop of the step: 4*d per (query
+    # row, prefix or tree key) pair; its compulsory bytes are the prefix and tree K/V and
+    # the queries
     rows = w.batch * w.tree_size * w.num_q_heads
-    prefix_flops = 4 * w.head_dim * w.tree_size * w.num_q_heads * total_L
-    prefix_bytes = 4 * total_L * w.num_kv_heads * w.head_dim + 2 * rows * w.head_dim
     kv_bytes = 4 * total_L * w.num_kv_heads * w.head_dim
+    partials_flops = step_flops
+    partials_bytes = kv_bytes + 4 * w.batch * w.tree_size * w.num_kv_heads * w.head_dim + 2 * rows * w.head_dim
     return dict(total_L=total_L, step_bytes=step_bytes, step_flops=step_flops,
-                prefix_flops=prefix_flops, prefix_bytes=prefix_bytes, kv_bytes=kv_bytes, rows=rows)
+                partials_flops=partials_flops, partials_bytes=partials_bytes, kv_bytes=kv_bytes, rows=rows)
 
 
 def config_of(inp, l2_note):
@@ -162,7 +163,7 @@ def kernel_source_hash():
 
 
 def recorded_traffic(workload_name):
-    """DRAM bytes per launch of the prefix kernel from the committed ncu summary, when it
+    """DRAM bytes per launch of the partials kernel from the committed ncu summary, when it
     was taken on the current kernel sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -267,11 +268,11 @@ def run_ours(args):
     ptr = {k: v.data_ptr() for k, v in d_in.items()}
     dims, ws, wsb = op.dims, op.workspace.data_ptr(), op.ws_bytes
 
-    def prefix():
-        rc = binding.call_prefix_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["cu"], dims, ws,
-                                     wsb, sp)
+    def partials():
+        rc = binding.call_partials_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["k_tree"], ptr["v_tree"],
+                                       ptr["parent"], ptr["cu"], dims, ws, wsb, sp)
         if rc:
-            raise binding.LSError(rc, "ls_verify_attn_prefix")
+            raise binding.LSError(rc, "ls_verify_attn_partials")
 
     def full_call():
         rc = binding.call_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["k_tree"], ptr["v_tree"],
@@ -286,7 +287,7 @@ def run_ours(args):
         flush.zero_()
         full_call()
         flush.zero_()
-        prefix()
+        partials()
     torch.cuda.synchronize(dev)
     st = op.check()
     if st != 0:
@@ -304,7 +305,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     with sampler:
-        # timed steps: one ls_verify_attn call each (prefix kernel + tree/combine kernel,
+        # timed steps: one ls_verify_attn call each (partials kernel + combine kernel,
         # the second launched as a programmatic dependent of the first)
         for k in range(K):
             flush.zero_()
@@ -317,16 +318,16 @@ def run_ours(args):
             flush.zero_()
             torch.cuda._sleep(spin_cycles)
             evp[k][0].record(stream)
-            prefix()
+            partials()
             evp[k][1].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    prefix_ms = [e[0].elapsed_time(e[1]) for e in evp]
+    partials_ms = [e[0].elapsed_time(e[1]) for e in evp]
     ms_per_step = float(statistics.mean(step_ms))
-    prefix_avg_ms = float(statistics.mean(prefix_ms))
-    ms_per_step, prefix_avg_ms = max_over_ranks([ms_per_step, prefix_avg_ms], device=dev)
+    partials_avg_ms = float(statistics.mean(partials_ms))
+    ms_per_step, partials_avg_ms = max_over_ranks([ms_per_step, partials_avg_ms], device=dev)
     st = op.check()
     if st != 0:
         raise binding.LSError(st, "device status after timing")
@@ -370,20 +371,20 @@ def run_ours(args):
     peaks, peak_kind = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    prefix_s = prefix_avg_ms / 1000.0
-    t_bytes = fig["prefix_bytes"] / (hbm * 1e9)
-    t_flops = fig["prefix_flops"] / (tc * 1e12)
+    part_s = partials_avg_ms / 1000.0
+    t_bytes = fig["partials_bytes"] / (hbm * 1e9)
+    t_flops = fig["partials_flops"] / (tc * 1e12)
     if t_flops >= t_bytes:
-        roof = {"bound": "tensor", "achieved": fig["prefix_flops"] / prefix_s / 1e12, "peak": tc,
+        roof = {"bound": "tensor", "achieved": fig["partials_flops"] / part_s / 1e12, "peak": tc,
                 "unit": "TFLOP/s"}
     else:
-        roof = {"bound": "hbm", "achieved": fig["prefix_bytes"] / prefix_s / 1e9, "peak": hbm,
+        roof = {"bound": "hbm", "achieved": fig["partials_bytes"] / part_s / 1e9, "peak": hbm,
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(w.name)
-    roof["kernel"] = "prefix (ls_verify_attn_prefix)"
+    roof["kernel"] = "partials (ls_verify_attn_partials: prefix and tree blocks)"
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured" else "fallback"
-    roof["kernel_us"] = prefix_avg_ms * 1000.0
+    roof["kernel_us"] = partials_avg_ms * 1000.0
     step_s = ms_per_step / 1000.0
     roof_step_s = max(fig["step_bytes"] / (hbm * 1e9), fig["step_flops"] / (tc * 1e12))
 
@@ -397,8 +398,8 @@ def run_ours(args):
             "roofline_step": {"roofline_us": roof_step_s * 1e6, "frac": roof_step_s / step_s,
                               "bytes": fig["step_bytes"], "flops": fig["step_flops"]},
             "roofline": roof, "gpu_launches": 2 * K, "plan": op.plan,
-            "kernel_timing": "prefix kernel timed in K further prefix-only launches after the K steps, "
-                             "same L2 flush and queueing",
+            "kernel_timing": "partials kernel timed in K further partials-only launches after the K "
+                             "steps, same L2 flush and queueing",
             "clocks": sampler.summary(), "e2e": e2e}
     if world == 1 and not args.no_cpu_baseline:
         us, n, dt, cores = time_oracle(inp, target_s=args.cpu_seconds)

@@ -118,29 +118,32 @@ LS_API int ls_verify_attn(const void* q, const void* k_cache, const void* v_cach
  * the caller ordering them), with the same dims and workspace; together they are
  * exactly ls_verify_attn. Arguments as for ls_verify_attn.
  *
- * ls_verify_attn_prefix (the "Cached-Teil" of section 2C): attention of every tree
- * query over its sequence's cached prefix with no mask. The prefix is split into
- * chunks of 128-key blocks; each chunk leaves a partial (out normalised by its own
- * sum, lse) in the workspace.
+ * ls_verify_attn_partials (the "Cached-Teil" and "Speculative-Teil" of section 2C):
+ * the keys of sequence b are its ceil(L_b/128) prefix blocks followed by one block of
+ * its T tree keys. They are split into chunks of consecutive blocks, and each chunk
+ * leaves, for every query row of one kv head's unit of rows, its partial (out
+ * normalised by its own sum, lse) in the workspace. Prefix keys are attended with no
+ * mask; a tree key is visible to node i when it is i or one of i's ancestors
+ * (tree_parent is checked: a bad tree is reported as LS_ERR_BAD_TREE by
+ * ls_verify_attn_check). k_cache and v_cache may be NULL when no sequence has a prefix
+ * (cu_seqlens_host all zero, or max_prefix_len = 0).
  *
- * ls_verify_attn_tree_combine (the "Speculative-Teil" and "Aggregation" of section
- * 2C): builds each node's ancestor-or-self set from tree_parent, attends over those
- * tree keys, merges the result with every prefix partial by log-sum-exp, and writes
- * `out` and `lse`.
+ * ls_verify_attn_combine (the "Aggregation" of section 2C): merges every row's
+ * partials by log-sum-exp and writes `out` and `lse`.
  */
-LS_API int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cache,
-                                 const int32_t* cu_seqlens, const ls_verify_dims* dims,
-                                 void* workspace, size_t workspace_bytes, void* stream);
-LS_API int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const void* v_tree,
-                                       const int32_t* tree_parent, const int32_t* cu_seqlens,
-                                       void* out, float* lse, const ls_verify_dims* dims,
-                                       void* workspace, size_t workspace_bytes, void* stream);
+LS_API int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_cache,
+                                   const void* k_tree, const void* v_tree, const int32_t* tree_parent,
+                                   const int32_t* cu_seqlens, const ls_verify_dims* dims, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+LS_API int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* lse,
+                                  const ls_verify_dims* dims, void* workspace, size_t workspace_bytes,
+                                  void* stream);
 
 /*
  * ls_verify_attn without a workspace argument, for callers that cannot allocate device
  * memory (the LongSpec pages have no counterpart: this is an interface convenience).
  *
- * ls_verify_attn needs caller-provided scratch for the prefix partials. A caller that
+ * ls_verify_attn needs caller-provided scratch for the attention partials. A caller that
  * only ever receives its input and output buffers, such as an operator plugin inside an
  * inference engine that owns the whole device heap and hands its plugins no allocator,
  * has no way to provide it. This call instead uses a fixed 32 MiB array that lives in
@@ -176,10 +179,10 @@ LS_API const char* ls_status_string(int status);
 
 /*
  * Describes how ls_verify_attn splits the work for these dims on the current device:
- * number of prefix work units (CTAs of the prefix kernel), 128-key blocks per unit,
- * and CTAs of the tree/combine kernel. Any pointer may be NULL. Returns a status.
+ * number of chunks (CTAs of the partials kernel), key blocks per chunk, and CTAs of
+ * the combine kernel. Any pointer may be NULL. Returns a status.
  */
-LS_API int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* prefix_ctas,
+LS_API int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* partials_ctas,
                         int32_t* blocks_per_chunk, int32_t* combine_ctas);
 
 #ifdef __cplusplus

@@ -1,6 +1,7 @@
-// Host-side check of the chunk plan: every (sequence, kv head, unit, 128-key
-// block) of the prefix is covered by exactly one chunk, chunk ids are dense, and the
-// per-sequence chunk ranges that the combine kernel uses agree with locate_chunk.
+// Host-side check of the chunk plan: every (sequence, kv head, unit, key block) is
+// covered by exactly one chunk, where the key blocks of a sequence are its 128-key
+// prefix blocks followed by its tree block; chunk ids are dense, and the per-sequence
+// chunk ranges that the combine kernel uses agree with locate_chunk.
 // Usage: plan_check B Hq Hkv T C uniform_n L_0 ... L_{B-1}   (exit 0 = pass)
 #include <cstdio>
 #include <cstdlib>
@@ -39,17 +40,20 @@ int main(int argc, char** argv) {
     const int expect = f + (c.kh * p.rg + c.rgi) * n + c.split;
     if (expect != cid) { printf("chunk %d: combine index %d\n", cid, expect); return 1; }
     if (c.key_end > c.key_begin && c.key_begin % ls::kBlockN) { printf("chunk %d unaligned start\n", cid); return 1; }
-    if (c.key_end - c.key_begin > p.C * ls::kBlockN) { printf("chunk %d too long\n", cid); return 1; }
+    const int nblk = ls::ceil_div(c.key_end - c.key_begin, ls::kBlockN) + (c.has_tree ? 1 : 0);
+    if (nblk > p.C) { printf("chunk %d too long\n", cid); return 1; }
     if (c.seq_offset != cu[c.b]) return 1;
     for (int k = c.key_begin; k < c.key_end; k += ls::kBlockN)
       seen[std::make_tuple(c.b, c.kh, c.rgi, k / ls::kBlockN)]++;
+    // the tree block is block number prefix_blocks(L) of the sequence's list
+    if (c.has_tree) seen[std::make_tuple(c.b, c.kh, c.rgi, ls::prefix_blocks(cu[c.b + 1] - cu[c.b]))]++;
   }
   if (ls::locate_chunk(p, cu.data(), total).valid) { printf("chunk past the end is valid\n"); return 1; }
   for (int b = 0; b < p.B; ++b) {
     const int L = cu[b + 1] - cu[b];
     for (int kh = 0; kh < p.Hkv; ++kh)
       for (int r = 0; r < p.rg; ++r)
-        for (int k = 0; k < ls::ceil_div(L, ls::kBlockN); ++k) {
+        for (int k = 0; k <= ls::prefix_blocks(L); ++k) {
           auto it = seen.find(std::make_tuple(b, kh, r, k));
           if (it == seen.end() || it->second != 1) {
             printf("block (%d,%d,%d,%d) covered %d times\n", b, kh, r, k,

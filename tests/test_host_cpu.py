@@ -30,13 +30,20 @@ def plan_check(tmp_path_factory):
     (1, 4, 1, 16, 3, -1, [1024]),
     (8, 32, 8, 64, 40, -1, [4096, 32768, 5000, 1, 0, 128, 129, 20000]),
     (3, 6, 3, 5, 2, -1, [0, 0, 0]),
-    (4, 8, 2, 33, 5, 3, [1200, 17, 0, 1920]),   # uniform plan: max 1920 -> 15 blocks -> 3 chunks of 5
-    (2, 64, 1, 128, 1, -1, [300, 1]),            # 8192 rows per kv head: 32 row groups
+    (4, 8, 2, 33, 5, 4, [1200, 17, 0, 1920]),   # uniform plan: max 1920 -> 15 prefix + 1 tree block -> 4 chunks of 5
+    (2, 64, 1, 128, 1, -1, [300, 1]),            # g = 64: 4 nodes per unit, 32 units per kv head
 ])
 def test_chunk_plan_covers_every_block_once(plan_check, B, Hq, Hkv, T, C, uniform, lengths):
     r = subprocess.run([plan_check, str(B), str(Hq), str(Hkv), str(T), str(C), str(uniform),
                         *map(str, lengths)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_plan_check_catches_an_uncovered_tree_block(plan_check):
+    # uniform plan of 3 chunks of 5 blocks: 1920 keys need 15 prefix blocks and the tree
+    # block, 16 in all, so the tree block of that sequence is left out
+    r = subprocess.run([plan_check, "1", "4", "1", "16", "5", "3", "1920"], capture_output=True, text=True)
+    assert r.returncode == 1 and "covered 0 times" in r.stdout
 
 
 def test_random_plans(plan_check):

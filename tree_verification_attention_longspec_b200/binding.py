@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "lib", "libls_verify_attn.so")
 LS_OK = 0
 STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3: "LS_ERR_WORKSPACE",
                 4: "LS_ERR_CUDA", 5: "LS_ERR_BAD_TREE", 6: "LS_ERR_TIMEOUT", 7: "LS_ERR_LENGTHS"}
-EXPORTED = ("ls_verify_attn", "ls_verify_attn_prefix", "ls_verify_attn_tree_combine",
+EXPORTED = ("ls_verify_attn", "ls_verify_attn_partials", "ls_verify_attn_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
             "ls_verify_attn_plan", "ls_verify_attn_static")
 
@@ -59,10 +59,10 @@ def load_library(path: str = LIB_PATH):
     P, D = ctypes.c_void_p, ctypes.POINTER(Dims)
     lib.ls_verify_attn.argtypes = [P, P, P, P, P, P, P, P, P, D, P, ctypes.c_size_t, P]
     lib.ls_verify_attn.restype = ctypes.c_int
-    lib.ls_verify_attn_prefix.argtypes = [P, P, P, P, D, P, ctypes.c_size_t, P]
-    lib.ls_verify_attn_prefix.restype = ctypes.c_int
-    lib.ls_verify_attn_tree_combine.argtypes = [P, P, P, P, P, P, P, D, P, ctypes.c_size_t, P]
-    lib.ls_verify_attn_tree_combine.restype = ctypes.c_int
+    lib.ls_verify_attn_partials.argtypes = [P, P, P, P, P, P, P, D, P, ctypes.c_size_t, P]
+    lib.ls_verify_attn_partials.restype = ctypes.c_int
+    lib.ls_verify_attn_combine.argtypes = [P, P, P, D, P, ctypes.c_size_t, P]
+    lib.ls_verify_attn_combine.restype = ctypes.c_int
     lib.ls_verify_attn_static.argtypes = [P, P, P, P, P, P, P, P, P, D, P]
     lib.ls_verify_attn_static.restype = ctypes.c_int
     lib.ls_verify_attn_workspace_size.argtypes = [D]
@@ -104,7 +104,7 @@ def plan(dims: Dims):
                                             ctypes.byref(c))
     if rc != LS_OK:
         raise LSError(rc, "ls_verify_attn_plan")
-    return {"prefix_ctas": a.value, "blocks_per_chunk": b.value, "combine_ctas": c.value}
+    return {"partials_ctas": a.value, "blocks_per_chunk": b.value, "combine_ctas": c.value}
 
 
 def call_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, out, lse, dims: Dims,
@@ -123,18 +123,18 @@ def call_static_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, out
                                                     cu_seqlens, out, lse, ctypes.byref(dims), stream))
 
 
-def call_prefix_raw(q, k_cache, v_cache, cu_seqlens, dims: Dims, workspace, workspace_bytes: int,
-                    stream) -> int:
-    return int(load_library().ls_verify_attn_prefix(q, k_cache, v_cache, cu_seqlens,
-                                                    ctypes.byref(dims), workspace, workspace_bytes,
-                                                    stream))
+def call_partials_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, dims: Dims, workspace,
+                      workspace_bytes: int, stream) -> int:
+    """ls_verify_attn_partials (the dominant kernel) on raw device addresses."""
+    return int(load_library().ls_verify_attn_partials(q, k_cache, v_cache, k_tree, v_tree, parent,
+                                                      cu_seqlens, ctypes.byref(dims), workspace,
+                                                      workspace_bytes, stream))
 
 
-def call_tree_combine_raw(q, k_tree, v_tree, parent, cu_seqlens, out, lse, dims: Dims, workspace,
-                          workspace_bytes: int, stream) -> int:
-    return int(load_library().ls_verify_attn_tree_combine(q, k_tree, v_tree, parent, cu_seqlens,
-                                                          out, lse, ctypes.byref(dims), workspace,
-                                                          workspace_bytes, stream))
+def call_combine_raw(cu_seqlens, out, lse, dims: Dims, workspace, workspace_bytes: int, stream) -> int:
+    """ls_verify_attn_combine on raw device addresses."""
+    return int(load_library().ls_verify_attn_combine(cu_seqlens, out, lse, ctypes.byref(dims), workspace,
+                                                     workspace_bytes, stream))
 
 
 def check(dims: Dims, workspace_ptr: int, stream_ptr: int) -> int:

@@ -59,8 +59,9 @@ int check_dims(const ls_verify_dims* d) {
 }
 
 // Chooses the chunk length C (in 128-key blocks) that minimises the estimated time of
-// the prefix kernel: waves of `slots` CTAs, each wave as long as its longest chunk
-// plus a fixed per-chunk cost for loading Q and writing the partial.
+// the partials kernel: waves of `slots` CTAs, each wave as long as its longest chunk
+// plus a fixed per-chunk cost for loading Q and writing the partial. A sequence's key
+// list is its prefix blocks plus one tree block.
 int make_plan(const ls_verify_dims* d, Plan* p) {
   int rc = check_dims(d);
   if (rc != LS_OK) return rc;
@@ -82,20 +83,20 @@ int make_plan(const ls_verify_dims* d, Plan* p) {
   q.rg = ls::ceil_div(q.T, q.tpu);
   q.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)q.d);
   q.scale_log2 = (float)((double)q.scale * 1.4426950408889634074);
-  q.n_combine = q.B * q.T * q.Hkv;
+  q.n_combine = (int32_t)(((long long)q.B * q.T * q.Hq + ls::kMergeRows - 1) / ls::kMergeRows);
 
   std::vector<int32_t> blocks(q.B);
   int32_t max_blocks = 0;
   for (int b = 0; b < q.B; ++b) {
     const int32_t L = d->cu_seqlens_host ? d->cu_seqlens_host[b + 1] - d->cu_seqlens_host[b]
                                          : d->max_prefix_len;
-    blocks[b] = ls::ceil_div(L, ls::kBlockN);
+    blocks[b] = ls::prefix_blocks(L) + 1;  // prefix blocks and the tree block
     if (blocks[b] > max_blocks) max_blocks = blocks[b];
   }
   const long long units = (long long)q.Hkv * q.rg;
   const long long slots = sms;  // one prefix CTA per SM
   const long long overhead = 2;  // per-chunk cost in blocks (Q load, partial store)
-  int32_t best_C = max_blocks > 0 ? max_blocks : 1;
+  int32_t best_C = max_blocks;
   long long best_cost = -1, best_n = 0;
   for (int32_t C = 1; C <= max_blocks; ++C) {
     long long n = 0;
@@ -112,7 +113,7 @@ int make_plan(const ls_verify_dims* d, Plan* p) {
   if (d->cu_seqlens_host) {
     q.uniform_n = -1;
   } else {
-    q.uniform_n = max_blocks > 0 ? ls::ceil_div(max_blocks, q.C) : 0;
+    q.uniform_n = ls::ceil_div(max_blocks, q.C);
   }
   long long n = 0;
   for (int b = 0; b < q.B; ++b)
@@ -140,36 +141,46 @@ size_t ls_verify_attn_workspace_size(const ls_verify_dims* dims) {
   return (size_t)ls::make_layout(p).total;
 }
 
-int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* prefix_ctas, int32_t* blocks_per_chunk,
+int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* partials_ctas, int32_t* blocks_per_chunk,
                         int32_t* combine_ctas) {
   Plan p;
   const int rc = make_plan(dims, &p);
   if (rc != LS_OK) return rc;
-  if (prefix_ctas) *prefix_ctas = p.n_chunks;
+  if (partials_ctas) *partials_ctas = p.n_chunks;
   if (blocks_per_chunk) *blocks_per_chunk = p.C;
   if (combine_ctas) *combine_ctas = p.n_combine;
   return LS_OK;
 }
 
-int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cache,
-                          const int32_t* cu_seqlens, const ls_verify_dims* dims, void* workspace,
-                          size_t workspace_bytes, void* stream) {
+int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree,
+                            const void* v_tree, const int32_t* tree_parent, const int32_t* cu_seqlens,
+                            const ls_verify_dims* dims, void* workspace, size_t workspace_bytes, void* stream) {
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != LS_OK) return rc;
-  if (q == nullptr || cu_seqlens == nullptr || !aligned16(q) || !aligned4(cu_seqlens))
+  const void* ptrs16[] = {q, k_tree, v_tree};
+  for (const void* x : ptrs16)
+    if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
+  if (tree_parent == nullptr || cu_seqlens == nullptr || !aligned4(tree_parent) || !aligned4(cu_seqlens))
     return LS_ERR_INVALID_ARG;
-  if (p.n_chunks > 0 && (k_cache == nullptr || v_cache == nullptr || !aligned16(k_cache) ||
-                         !aligned16(v_cache)))
-    return LS_ERR_INVALID_ARG;
+  if (k_cache == nullptr || v_cache == nullptr || !aligned16(k_cache) || !aligned16(v_cache)) {
+    // a call without prefix keys may pass null caches
+    const bool any_prefix = dims->cu_seqlens_host ? dims->cu_seqlens_host[dims->batch] > 0 : dims->max_prefix_len > 0;
+    if (any_prefix || (k_cache != nullptr && !aligned16(k_cache)) || (v_cache != nullptr && !aligned16(v_cache)))
+      return LS_ERR_INVALID_ARG;
+  }
   const ls::Layout lay = ls::make_layout(p);
   if (!workspace_ok(workspace, workspace_bytes, lay)) return LS_ERR_WORKSPACE;
   char* ws = static_cast<char*>(workspace);
   (void)cudaGetLastError();  // clear a stale, non-sticky error from unrelated work
-  ls::PrefixArgs pa;
+  ls::PartialsArgs pa;
   pa.q = static_cast<const uint16_t*>(q);
-  pa.k_cache = static_cast<const uint16_t*>(k_cache);
-  pa.v_cache = static_cast<const uint16_t*>(v_cache);
+  // the tensor maps need an address even where no prefix row is ever read
+  pa.k_cache = static_cast<const uint16_t*>(k_cache ? k_cache : k_tree);
+  pa.v_cache = static_cast<const uint16_t*>(v_cache ? v_cache : v_tree);
+  pa.k_tree = static_cast<const uint16_t*>(k_tree);
+  pa.v_tree = static_cast<const uint16_t*>(v_tree);
+  pa.parent = tree_parent;
   pa.cu = cu_seqlens;
   pa.o_part = reinterpret_cast<float*>(ws + lay.o_part);
   pa.lse_part = reinterpret_cast<float*>(ws + lay.lse_part);
@@ -177,35 +188,26 @@ int ls_verify_attn_prefix(const void* q, const void* k_cache, const void* v_cach
   pa.p = p;
   // rows of the K/V tensors that the TMA descriptors may address (an upper bound is
   // enough: no block is ever read past its sequence's end)
-  const int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
-                                                : (int64_t)dims->batch * dims->max_prefix_len;
-  const cudaError_t e = ls::launch_prefix_tc(pa, kv_rows, static_cast<cudaStream_t>(stream));
+  int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
+                                          : (int64_t)dims->batch * dims->max_prefix_len;
+  if (k_cache == nullptr) kv_rows = (int64_t)p.B * p.T;
+  const cudaError_t e = ls::launch_partials(pa, kv_rows, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
 }
 
-int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const void* v_tree,
-                                const int32_t* tree_parent, const int32_t* cu_seqlens, void* out,
-                                float* lse, const ls_verify_dims* dims, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims,
+                           void* workspace, size_t workspace_bytes, void* stream) {
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != LS_OK) return rc;
-  const void* ptrs16[] = {q, k_tree, v_tree, out};
-  for (const void* x : ptrs16)
-    if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
-  const void* ptrs4[] = {tree_parent, cu_seqlens, lse};
-  for (const void* x : ptrs4)
-    if (x == nullptr || !aligned4(x)) return LS_ERR_INVALID_ARG;
+  if (out == nullptr || !aligned16(out)) return LS_ERR_INVALID_ARG;
+  if (cu_seqlens == nullptr || lse == nullptr || !aligned4(cu_seqlens) || !aligned4(lse)) return LS_ERR_INVALID_ARG;
   const ls::Layout lay = ls::make_layout(p);
   if (!workspace_ok(workspace, workspace_bytes, lay)) return LS_ERR_WORKSPACE;
   char* ws = static_cast<char*>(workspace);
   (void)cudaGetLastError();
   ls::CombineArgs ca;
-  ca.q = static_cast<const uint16_t*>(q);
-  ca.k_tree = static_cast<const uint16_t*>(k_tree);
-  ca.v_tree = static_cast<const uint16_t*>(v_tree);
-  ca.parent = tree_parent;
   ca.cu = cu_seqlens;
   ca.o_part = reinterpret_cast<const float*>(ws + lay.o_part);
   ca.lse_part = reinterpret_cast<const float*>(ws + lay.lse_part);
@@ -214,8 +216,7 @@ int ls_verify_attn_tree_combine(const void* q, const void* k_tree, const void* v
   ca.lse = lse;
   ca.status = reinterpret_cast<uint32_t*>(ws + lay.status);
   ca.p = p;
-  if (ls::launch_tree_combine(ca, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return LS_ERR_CUDA;
+  if (ls::launch_combine(ca, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
 }
 
@@ -227,17 +228,11 @@ int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache, cons
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != LS_OK) return rc;
-  const void* ptrs16[] = {q, k_tree, v_tree, out};
-  for (const void* x : ptrs16)
-    if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
-  const void* ptrs4[] = {tree_parent, cu_seqlens, lse};
-  for (const void* x : ptrs4)
-    if (x == nullptr || !aligned4(x)) return LS_ERR_INVALID_ARG;
-  rc = ls_verify_attn_prefix(q, k_cache, v_cache, cu_seqlens, dims, workspace, workspace_bytes,
-                             stream);
+  if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
+  rc = ls_verify_attn_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, workspace,
+                               workspace_bytes, stream);
   if (rc != LS_OK) return rc;
-  return ls_verify_attn_tree_combine(q, k_tree, v_tree, tree_parent, cu_seqlens, out, lse, dims,
-                                     workspace, workspace_bytes, stream);
+  return ls_verify_attn_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream);
 }
 
 int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void* stream) {

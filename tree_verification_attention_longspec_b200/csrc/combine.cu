@@ -1,0 +1,144 @@
+// Log-sum-exp combine of the attention partials.
+//
+// LongSpec, gist.science summary, section 2C ("Aggregation"): the partial results are
+// joined by a log-sum-exp step into one exact softmax. Every chunk of the partials
+// kernel left, for each row of its unit, its output normalised by its own sum (o_part)
+// and its lse in the log2 domain (lse_part); the chunks of one unit cover its prefix
+// blocks and its tree block once each. For a row with partials (o_x, l_x):
+//   M = max_x l_x,  w_x = 2^(l_x - M),  out = sum_x w_x o_x / sum_x w_x,
+//   lse = (M + log2 sum_x w_x) * ln 2   (natural log, scale included).
+// One warp per output row (tree node i of sequence b, query head h); lanes split the
+// head dimension. The kernel is launched as a programmatic dependent of the partials
+// kernel and waits for its results with griddepcontrol.wait. It uses no shared memory
+// beyond a status word, so one of its CTAs fits beside a partials CTA on an SM and is
+// ready when that grid ends.
+#include "ls_device.cuh"
+
+namespace ls {
+namespace {
+
+constexpr int kPrefetch = 16;  // partials in flight per warp
+
+template <int D>
+__global__ void __launch_bounds__(32 * kMergeRows) combine_kernel(CombineArgs a) {
+  constexpr int E = D / 32;  // head-dim elements per lane
+  const Plan& p = a.p;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ uint32_t err_s;
+  if (threadIdx.x == 0) err_s = 0u;
+  __syncthreads();
+  // the partials kernel may still be running: wait for its grid to finish
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  const int64_t n_rows = (int64_t)p.B * p.T * p.Hq;
+  const int64_t row = (int64_t)blockIdx.x * kMergeRows + warp;
+  uint32_t err = 0u;
+  if (row < n_rows) {
+    const int tok = (int)(row / p.Hq), h = (int)(row % p.Hq);
+    const int b = tok / p.T, i = tok % p.T;
+    const int kh = h / p.g, j = h % p.g;
+    int first = 0, n = 0, total = 0;
+    sequence_chunks(p, a.cu, b, &first, &n, &total);
+    const int32_t L = a.cu[b + 1] - a.cu[b];
+    // the device lengths must give the chunk grid the host planned (else some keys were
+    // never attended): same chunk count, and a uniform plan long enough for this L
+    const bool lengths_ok = L >= 0 && total == p.n_chunks &&
+                            (p.uniform_n < 0 || (int64_t)prefix_blocks(L) + 1 <= (int64_t)p.uniform_n * p.C);
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    float M = -INFINITY, Lsum = 0.f;  // running max of the lse and sum of weights 2^(l - M)
+    if (lengths_ok) {
+      int32_t u, rl;
+      unit_row(p, i, j, &u, &rl);
+      const int cbase = first + (kh * p.rg + u) * n;
+      for (int x0 = 0; x0 < n; x0 += kPrefetch) {
+        const int nx = min(kPrefetch, n - x0);
+        // every lane one chunk's lse and status; up to kPrefetch chunk outputs in flight
+        float lx = -INFINITY;
+        if (lane < nx) {
+          lx = a.lse_part[(size_t)(cbase + x0 + lane) * kUnitRows + rl];
+          err |= a.chunk_status[cbase + x0 + lane];
+        }
+        float ov[kPrefetch][E];
+        const float* base = a.o_part + ((size_t)(cbase + x0) * kUnitRows + rl) * D + lane * E;
+#pragma unroll
+        for (int x = 0; x < kPrefetch; ++x) {
+          if (x < nx) {
+            const float* op = base + (size_t)x * kUnitRows * D;
+            if constexpr (E == 4) {
+              const float4 v = *reinterpret_cast<const float4*>(op);
+              ov[x][0] = v.x;
+              ov[x][1] = v.y;
+              ov[x][2] = v.z;
+              ov[x][3] = v.w;
+            } else {
+              const float2 v = *reinterpret_cast<const float2*>(op);
+              ov[x][0] = v.x;
+              ov[x][1] = v.y;
+            }
+          }
+        }
+        float mx = lx;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+        const float Mn = fmaxf(M, mx);
+        const float corr = M == Mn ? 1.f : exp2f(M - Mn);       // M = -inf before any weight: 0
+        const float wl = lx == -INFINITY ? 0.f : exp2f(lx - Mn);  // this lane's chunk weight
+        Lsum = Lsum * corr + warp_sum(wl);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] *= corr;
+        M = Mn;
+#pragma unroll
+        for (int x = 0; x < kPrefetch; ++x) {
+          const float w = __shfl_sync(0xffffffffu, wl, x);
+          if (x < nx && w > 0.f) {  // an empty chunk leaves its output slot unwritten
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = fmaf(w, ov[x][e], acc[e]);
+          }
+        }
+      }
+    } else {
+      err |= kErrLengths;
+    }
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    uint16_t* dst = a.out + row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      const uint32_t lo = f32_to_bf16(acc[e] * inv), hi = f32_to_bf16(acc[e + 1] * inv);
+      *reinterpret_cast<uint32_t*>(dst + e) = lo | (hi << 16);
+    }
+    if (lane == 0) a.lse[row] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+  }
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o2);
+  if (lane == 0 && err) atomicOr(&err_s, err);
+  __syncthreads();
+  if (threadIdx.x == 0) a.status[blockIdx.x] = err_s;
+}
+
+template <int D>
+cudaError_t launch_d(const CombineArgs& a, cudaStream_t stream) {
+  // a programmatic dependent of the partials kernel: its CTAs may be scheduled while
+  // that grid runs and wait in griddepcontrol.wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.p.n_combine);
+  cfg.blockDim = dim3(32 * kMergeRows);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel<D>, a);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
+  if (a.p.n_combine == 0) return cudaSuccess;
+  return a.p.d == 64 ? launch_d<64>(a, stream) : launch_d<128>(a, stream);
+}
+
+}  // namespace ls

@@ -9,10 +9,15 @@ namespace ls {
 
 constexpr float kLn2 = 0.693147180559945309417f;
 
-struct PrefixArgs {
+// The partials kernel: every chunk's prefix blocks and, for the chunk that holds it,
+// the masked tree block.
+struct PartialsArgs {
   const uint16_t* q;
   const uint16_t* k_cache;
   const uint16_t* v_cache;
+  const uint16_t* k_tree;
+  const uint16_t* v_tree;
+  const int32_t* parent;
   const int32_t* cu;
   float* o_part;
   float* lse_part;
@@ -20,11 +25,8 @@ struct PrefixArgs {
   Plan p;
 };
 
+// The combine kernel: the log-sum-exp merge of every chunk's partial.
 struct CombineArgs {
-  const uint16_t* q;
-  const uint16_t* k_tree;
-  const uint16_t* v_tree;
-  const int32_t* parent;
   const int32_t* cu;
   const float* o_part;
   const float* lse_part;
@@ -54,6 +56,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Launchers (defined in the kernel files, called by the host API).
 namespace ls {
-cudaError_t launch_prefix_tc(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream);
-cudaError_t launch_tree_combine(const CombineArgs& a, cudaStream_t stream);
+cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 }  // namespace ls

@@ -1,13 +1,16 @@
 // Work split and workspace layout shared by the host launcher and the kernels.
 //
-// The prefix ("Cached-Teil") work is cut into chunks. A chunk is one
-// (sequence b, kv head kh, unit u, key range) and becomes one CTA of the prefix
-// kernel. The query rows of a kv head are its T*g (tree node i, head-in-group j)
-// pairs; a unit holds the rows of tpu = floor(256 / g) consecutive tree nodes, so its
-// rows are whole nodes (at most 256 of them, row (i - u*tpu)*g + j of the unit) and
-// one TMA box brings them in. Every chunk of a sequence covers C consecutive 128-key
-// blocks (the last one fewer), so the chunk grid follows from the prefix lengths and
-// C alone, and the device recomputes it from cu_seqlens without any table in memory.
+// The attention work is cut into chunks. A chunk is one (sequence b, kv head kh, unit
+// u, range of key blocks) and becomes one CTA of the partials kernel. The query rows of
+// a kv head are its T*g (tree node i, head-in-group j) pairs; a unit holds the rows of
+// tpu = floor(256 / g) consecutive tree nodes, so its rows are whole nodes (at most 256
+// of them, row (i - u*tpu)*g + j of the unit) and one TMA box brings them in.
+// The keys of sequence b form ceil(L_b / 128) prefix blocks ("Cached-Teil", no mask)
+// followed by one block of its T <= 128 tree keys ("Speculative-Teil", tree mask).
+// Every chunk of a sequence covers C consecutive blocks of that list, so the chunk
+// that holds the tree block also attends the last prefix keys, and a sequence without
+// prefix still has one chunk. The chunk grid follows from the prefix lengths and C
+// alone, and the device recomputes it from cu_seqlens without any table in memory.
 #pragma once
 #include <stdint.h>
 
@@ -21,7 +24,8 @@ namespace ls {
 
 constexpr int kBlockN = 128;       // keys per block of the prefix loop
 constexpr int kUnitRows = 256;     // query rows per prefix chunk (two 128-row MMA tiles)
-constexpr int kMaxTree = 128;      // largest supported tree
+constexpr int kMaxTree = 128;      // largest supported tree (one key block)
+constexpr int kMergeRows = 4;      // output rows per CTA of the combine kernel (a warp each)
 
 // device-side status bits (combined into one LS_ERR_* by ls_verify_attn_check)
 constexpr uint32_t kErrBadTree = 1u;
@@ -35,19 +39,22 @@ struct Plan {
   int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
   int32_t C;           // 128-key blocks per chunk
   int32_t uniform_n;   // >= 0: chunks per unit for every sequence; -1: from L_b
-  int32_t n_chunks;    // prefix CTAs
-  int32_t n_combine;   // tree/combine CTAs = B * T * Hkv
+  int32_t n_chunks;    // partials-kernel CTAs
+  int32_t n_combine;   // combine CTAs = ceil(B * T * Hq / kMergeRows)
   float scale;         // softmax scale
   float scale_log2;    // softmax scale * log2(e)
 };
 
 LS_HD int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
 
-// chunks of one (sequence, kv head, unit) for a prefix of L keys
+// 128-key blocks of a prefix of L keys
+LS_HD int32_t prefix_blocks(int32_t L) { return L > 0 ? ceil_div(L, kBlockN) : 0; }
+
+// chunks of one (sequence, kv head, unit) for a prefix of L keys: its prefix blocks
+// and the tree block, C per chunk
 LS_HD int32_t chunks_per_unit(const Plan& p, int32_t L) {
   if (p.uniform_n >= 0) return p.uniform_n;
-  if (L <= 0) return 0;
-  return ceil_div(ceil_div(L, kBlockN), p.C);
+  return ceil_div(prefix_blocks(L) + 1, p.C);
 }
 
 // Unit and row inside the unit of query row (tree node i, head-in-group j).
@@ -58,8 +65,9 @@ LS_HD void unit_row(const Plan& p, int32_t i, int32_t j, int32_t* unit, int32_t*
 
 struct ChunkCoord {
   int32_t b, kh, rgi, split, n_split;  // sequence, kv head, unit, split index, splits of unit
-  int32_t key_begin, key_end;          // key range inside the sequence's prefix
+  int32_t key_begin, key_end;          // prefix key range of the chunk
   int32_t seq_offset;                  // cu_seqlens[b]
+  bool has_tree;                       // the chunk also attends the tree block
   bool valid;
 };
 
@@ -83,10 +91,12 @@ LS_HD ChunkCoord locate_chunk(const Plan& p, const int32_t* cu, int32_t cid) {
       c.n_split = n;
       c.seq_offset = cu[b];
       const int32_t Lc = L < 0 ? 0 : L;
-      int32_t kb = c.split * p.C * kBlockN;
-      int32_t ke = kb + p.C * kBlockN;
+      const int32_t v0 = c.split * p.C, v1 = v0 + p.C;  // blocks [v0, v1) of the key list
+      const int32_t kb = v0 * kBlockN, ke = v1 * kBlockN;
       c.key_begin = kb < Lc ? kb : Lc;
       c.key_end = ke < Lc ? ke : Lc;
+      const int32_t tree_block = prefix_blocks(Lc);
+      c.has_tree = v0 <= tree_block && tree_block < v1;
       c.valid = true;
       return c;
     }

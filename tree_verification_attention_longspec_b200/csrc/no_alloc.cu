@@ -1,7 +1,7 @@
 // ls_verify_attn_static: tree-verification attention for callers that cannot allocate
 // device memory.
 //
-// ls_verify_attn needs a caller-provided workspace for the prefix partials. Some
+// ls_verify_attn needs a caller-provided workspace for the attention partials. Some
 // callers only ever receive their input and output buffers and have no way to obtain
 // more device memory: for example an operator plugin running inside an inference
 // engine that owns the whole device heap and exposes no allocator to its plugins, or

@@ -1,12 +1,16 @@
-// Prefix partial attention on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
+// Attention partials on the 5th-generation tensor cores (tcgen05, TMEM, TMA).
 //
 // LongSpec, gist.science summary, section 2C: the cached prefix is attended with no
-// mask, and it carries most of the work, so it runs on the fastest path. With grouped-
-// query attention the T*g (tree node, head-in-group) rows of one kv head share every
-// key, so the prefix step is a dense contraction: S = Q K^T and O += P V. One CTA handles
-// one chunk: a 256-row unit of one (sequence, kv head), as two 128-row query tiles,
-// against a range of 128-key blocks, and leaves its partial (out normalised by its own
-// sum, lse in the log2 domain) for the combine kernel.
+// mask ("Cached-Teil"), the speculative tree tokens under the tree mask
+// ("Speculative-Teil"), and the partial results are joined by log-sum-exp
+// ("Aggregation"). With grouped-query attention the T*g (tree node, head-in-group) rows
+// of one kv head share every key, so each part is a dense contraction: S = Q K^T and
+// O += P V. One CTA handles one chunk: a 256-row unit of one (sequence, kv head), as two
+// 128-row query tiles, against a run of 128-key blocks; the chunk that ends the
+// sequence's key list also takes the block of its T <= 128 tree keys, with every score
+// outside the row's ancestor-or-self set masked. A masked block is one more step of the
+// same online softmax, which is the log-sum-exp join itself. The CTA leaves its partial
+// (out normalised by its own sum, lse in the log2 domain) for the combine kernel.
 //
 // Ping-pong. Each query tile t has one softmax warpgroup, one score buffer S_t and one
 // output accumulator O_t in TMEM. The MMA thread walks the key blocks and, per block j,
@@ -23,7 +27,8 @@
 //              is m raised and O_t rescaled in TMEM. P (bf16) overwrites the scores in
 //              two halves of 64 keys, each announced on its own barrier, so the MMA
 //              thread starts on the first half while the second is computed.
-//   warp 8     TMA producer: streams 128-key K and V blocks into a ring of slots.
+//   warp 8     TMA producer: Q, then 128-key K and V blocks (prefix, then tree) into a
+//              ring of slots.
 //   warp 9     MMA issuer (one thread): S = Q K^T (shared-memory operands, N = 128) and
 //              O += P V (P from TMEM, N = d), tcgen05.commit to mbarriers.
 // TMEM columns (512 allocated): S_t at 128 t, O_t at 256 + d t.
@@ -68,9 +73,11 @@ struct Cfg {
 
 struct alignas(64) TcParams {
   CUtensorMap tmap_q;
-  CUtensorMap tmap_k;
+  CUtensorMap tmap_k;   // prefix keys
   CUtensorMap tmap_v;
-  PrefixArgs a;
+  CUtensorMap tmap_kt;  // tree keys
+  CUtensorMap tmap_vt;
+  PartialsArgs a;
 };
 
 struct Bars {
@@ -82,11 +89,15 @@ struct Bars {
   uint64_t o_full[kTiles];     // every MMA of tile t finished
   uint32_t tmem_base;
   uint32_t abort;
+  uint32_t tree_err;          // a parent link that is not a rooted tree's
+  int16_t parent[kMaxTree];   // the sequence's tree (chunks that hold the tree block)
 };
 
-// The kernel asks for the whole dynamic window a CTA may have and aligns its layout up
-// to 1024 bytes inside it (the 128-byte swizzle atom repeats every 1024 bytes).
-constexpr int kSmemWindow = 232448;
+// The kernel asks for the dynamic window of a CTA less 1 KB (so that one CTA of the
+// combine kernel, which needs no shared memory beyond the 1 KB every CTA reserves, can
+// wait beside it) and aligns its layout up to 1024 bytes inside it (the 128-byte
+// swizzle atom repeats every 1024 bytes).
+constexpr int kSmemWindow = 232448 - 1024;
 template <int D>
 constexpr int smem_need() {
   return Cfg<D>::kBarOff + (int)sizeof(Bars) + 1024;
@@ -134,24 +145,71 @@ __device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float 
   }
 }
 
+// Tree mask (LongSpec, gist.science summary, section 2C, "Baum-Maskierung") on the
+// scores of the tree block in this thread's TMEM lane: key x (tree node x) stays visible
+// when x is the row's node or one of its ancestors, found by following parent links.
+// Every link is checked (node 0 is the root with parent -1, any other node's parent
+// lies below it), so the walk ends; a failed check raises `bad`. node < 0 (a padding
+// row) masks every key. The scores go back to TMEM as -inf where masked.
+__device__ __forceinline__ bool mask_tree_scores(const int16_t* parent, uint32_t tS, int node) {
+  uint32_t am[4] = {0u, 0u, 0u, 0u};
+  bool bad = false;
+  if (node >= 0) {
+    int x = node;
+    for (int step = 0; step <= kMaxTree; ++step) {
+      const uint32_t bit = 1u << (x & 31);
+      const int w = x >> 5;
+      am[0] |= w == 0 ? bit : 0u;
+      am[1] |= w == 1 ? bit : 0u;
+      am[2] |= w == 2 ? bit : 0u;
+      am[3] |= w == 3 ? bit : 0u;
+      const int pp = parent[x];
+      if (x == 0) {
+        bad = pp != -1;
+        break;
+      }
+      if (pp < 0 || pp >= x) {
+        bad = true;
+        break;
+      }
+      x = pp;
+    }
+  }
+  __syncwarp();  // the TMEM accesses below are warp-collective
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t r[32];
+    tmem_ld32(tS + 32 * q, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (!((am[q] >> e) & 1u)) r[e] = __float_as_uint(-INFINITY);
+    tmem_st32(tS + 32 * q, r);
+  }
+  tmem_wait_st();
+  return bad;
+}
+
 template <int D, int EMU>
-__global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_constant__ TcParams P) {
+__global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_constant__ TcParams P) {
   using C = Cfg<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
-  const PrefixArgs& a = P.a;
+  const PartialsArgs& a = P.a;
   const Plan& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const ChunkCoord c = locate_chunk(p, a.cu, blockIdx.x);
   if (!c.valid) return;  // more CTAs than the device lengths need: the combine reports it
   const int n_keys = c.key_end - c.key_begin;
-  const int nb = (n_keys + kBlockN - 1) / kBlockN;
-  const int tail_shift = nb * kBlockN - n_keys;  // masked leading columns of the last block
+  const int nb = (n_keys + kBlockN - 1) / kBlockN;  // prefix blocks
+  const int tail_shift = nb * kBlockN - n_keys;      // masked leading columns of the last one
+  const bool has_tree = c.has_tree;
+  const int nbt = nb + (has_tree ? 1 : 0);  // blocks, the tree block (block nb) last
   const int tok0 = c.rgi * p.tpu;                    // first tree node of the unit
   const int rows_here = min(p.tpu, p.T - tok0) * p.g;  // rows of the unit that exist
-  if (nb == 0) {  // empty key range: an empty partial
+  if (nbt == 0) {  // empty key range: an empty partial
     for (int r = tid; r < rows_here; r += kThreads) a.lse_part[(size_t)blockIdx.x * kUnitRows + r] = -INFINITY;
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
     return;
@@ -171,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
     mbar_init(&bars->o_full[0], 1);
     mbar_init(&bars->o_full[1], 1);
     bars->abort = 0u;
+    bars->tree_err = 0u;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -181,6 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
     tma_prefetch_map(&P.tmap_q);
     tma_prefetch_map(&P.tmap_k);
     tma_prefetch_map(&P.tmap_v);
+    if (has_tree) {
+      tma_prefetch_map(&P.tmap_kt);
+      tma_prefetch_map(&P.tmap_vt);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -204,9 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
                     c.b * p.T + tok0);
       int issued = 0, slot = 0, use = 0;
       bool ok = true;
-      for (int j = 0; j < nb && ok; ++j) {
-        int key0 = c.key_begin + j * kBlockN;
-        if (j == nb - 1) key0 -= tail_shift;  // the box ends at the sequence end
+      for (int j = 0; j < nbt && ok; ++j) {
+        // prefix block j, or the tree block: the sequence's T nodes (the rows after them
+        // belong to the next sequence or lie past the tensor, read as zeros; masked)
+        const bool tree = j == nb;
+        int row = c.seq_offset + c.key_begin + j * kBlockN;
+        if (j == nb - 1) row -= tail_shift;  // the box ends at the sequence end
+        if (tree) row = c.b * p.T;
         for (int kv = 0; kv < 2; ++kv) {
           if (!mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs)) {
             ok = false;
@@ -214,10 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
           }
           mbar_arrive_expect_tx(&bars->full[slot], C::kTileBytes);
           uint8_t* dst = smem + C::kSlotOff + slot * C::kTileBytes;
-          const CUtensorMap* map = kv ? &P.tmap_v : &P.tmap_k;
+          const CUtensorMap* map = tree ? (kv ? &P.tmap_vt : &P.tmap_kt) : (kv ? &P.tmap_v : &P.tmap_k);
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, c.seq_offset + key0);
+            tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
           ++issued;
           if (++slot == C::kSlots) {
             slot = 0;
@@ -251,8 +318,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
             make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
+      // the tree of the sequence, for the tree mask; a parent outside [-1, T) is stored
+      // as a value that fails the walk's checks
+      if (has_tree) {
+        for (int x = tid; x < p.T; x += 256) {
+          const int32_t pp = a.parent[(size_t)c.b * p.T + x];
+          bars->parent[x] = (int16_t)(pp >= -1 && pp < p.T ? pp : kMaxTree);
+        }
+      }
     }
-    // the padding is in shared memory: warps 0-7 and the MMA warp meet at barrier 1
+    // the padding and the tree are in shared memory: warps 0-7 and the MMA warp meet at
+    // barrier 1
     if (warp < 8 || warp == kMmaWarp) asm volatile("bar.sync 1, 288;" ::: "memory");
 
     if (warp == kMmaWarp) {
@@ -311,10 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
           umma_commit(&bars->empty[slot]);
           advance();
         }
-        for (int j = 0; j < nb && ok; ++j) {
+        for (int j = 0; j < nbt && ok; ++j) {
           const int sv = slot, uv = use;  // V(j)
           advance();
-          const bool more = j + 1 < nb;
+          const bool more = j + 1 < nbt;
           const int sk = slot, uk = use;  // K(j+1), when there is one
           const uint32_t pp = j & 1;
           ok = wait(&bars->full[sv], uv);
@@ -353,16 +429,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
       const uint32_t tO = tbase + lane_base + C::kColO + t * D;
       const float cs = p.scale_log2;
       float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
+      const int ur = t * 128 + row;       // row of the unit
+      const bool has_row = ur < rows_here;
+      const int node = tok0 + ur / p.g;   // its tree node
       bool ok = true;
-      for (int j = 0; j < nb; ++j) {
+      for (int j = 0; j < nbt; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], j & 1, abort, kTimeoutNs));
         if (!ok) break;
         tc_fence_after_sync();
+        const int shift = j == nb - 1 ? tail_shift : 0;  // masked leading columns
+        const bool tree_blk = j == nb;                      // keys = the sequence's tree nodes
+        if (tree_blk && mask_tree_scores(bars->parent, tS, has_row ? node : -1)) bars->tree_err = 1u;
         // All 128 scores for the row maximum; the scores of keys 0..63 stay in registers
         // for P's first half, those of keys 64..127 are read again for the second half.
         float lo[kHalf];
         float mx;
-        const int shift = j == nb - 1 ? tail_shift : 0;  // masked leading columns
         {
           uint32_t r[4][32];
 #pragma unroll
@@ -395,13 +476,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
         const bool raise = mx > m + kRescaleThreshold;
         const bool any_raise = __any_sync(0xffffffffu, raise);
         // masked columns (-inf) and the rare blocks that raise m take the MUFU-only path
-        const bool mufu_only = EMU == 0 || shift > 0 || any_raise;
+        const bool mufu_only = EMU == 0 || shift > 0 || tree_blk || any_raise;
         const float m_new = raise ? mx : m;
+        // a row that has seen no visible key yet (a padding row of a tree-only chunk)
+        // keeps m = -inf; its P is 0 against any finite reference
+        const float m_ref = m_new == -INFINITY ? 0.f : m_new;
         float sum0 = 0.f, sum1 = 0.f;
         {
           uint32_t pk[kHalf / 2];
-          if (mufu_only) make_p<0>(lo, cs, m_new, pk, sum0, sum1);
-          else make_p<EMU>(lo, cs, m_new, pk, sum0, sum1);
+          if (mufu_only) make_p<0>(lo, cs, m_ref, pk, sum0, sum1);
+          else make_p<EMU>(lo, cs, m_ref, pk, sum0, sum1);
           if (any_raise) {
             // the maximum moved up: rescale what O_t and l hold. O_t is idle: every PV of
             // this tile issued before S_t(j) has completed (s_full), and PV_t(j) waits for
@@ -442,8 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
         }
         {
           uint32_t pk[kHalf / 2];
-          if (mufu_only) make_p<0>(hi, cs, m, pk, sum0, sum1);
-          else make_p<EMU>(hi, cs, m, pk, sum0, sum1);
+          if (mufu_only) make_p<0>(hi, cs, m_ref, pk, sum0, sum1);
+          else make_p<EMU>(hi, cs, m_ref, pk, sum0, sum1);
           tmem_st32(tS + 32, pk);  // keys 64..127 -> columns 32..63
           tmem_wait_st();
           tc_fence_before_sync();
@@ -509,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefix_tc_kernel(const __grid_con
     tc_fence_after_sync();
     tmem_dealloc(tbase, C::kTmemCols);
   }
-  if (tid == 0) a.chunk_status[blockIdx.x] = bars->abort ? kErrTimeout : 0u;
+  if (tid == 0) a.chunk_status[blockIdx.x] = (bars->abort ? kErrTimeout : 0u) | (bars->tree_err ? kErrBadTree : 0u);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -554,11 +638,14 @@ bool make_q_map(CUtensorMap* map, const void* base, int D, const Plan& p) {
 }
 
 template <int D, int EMU>
-cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) {
+cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream) {
   TcParams P;
   P.a = a;
+  const int64_t tree_rows = (int64_t)a.p.B * a.p.T;
   if (!make_q_map(&P.tmap_q, a.q, D, a.p) || !make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows) ||
-      !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows))
+      !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows) ||
+      !make_kv_map(&P.tmap_kt, a.k_tree, D, a.p.Hkv, tree_rows) ||
+      !make_kv_map(&P.tmap_vt, a.v_tree, D, a.p.Hkv, tree_rows))
     return cudaErrorInvalidValue;
   const int smem = kSmemWindow;
   // opt in to the large shared-memory carve-out once per device
@@ -566,17 +653,17 @@ cudaError_t launch_d(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) 
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(prefix_tc_kernel<D, EMU>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(partials_tc_kernel<D, EMU>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  prefix_tc_kernel<D, EMU><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
+  partials_tc_kernel<D, EMU><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefix_tc(const PrefixArgs& a, int64_t kv_rows, cudaStream_t stream) {
+cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream) {
   if (a.p.n_chunks == 0) return cudaSuccess;
   // One pair of scores in four takes the FMA-pipe exponential: a quarter of the
   // softmax's exponentials move off the special-function unit (MUFU), which is as busy
