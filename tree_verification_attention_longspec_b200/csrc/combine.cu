@@ -17,41 +17,50 @@
 namespace ls {
 namespace {
 
-constexpr int kPrefetch = 16;  // partials in flight per warp
+constexpr int kPrefetch = 20;  // partials in flight per warp (the headline has 18 per row)
 
 template <int D>
-__global__ void __launch_bounds__(32 * kMergeRows) combine_kernel(CombineArgs a) {
+__global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   constexpr int E = D / 32;  // head-dim elements per lane
   const Plan& p = a.p;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   __shared__ uint32_t err_s;
   if (threadIdx.x == 0) err_s = 0u;
   __syncthreads();
-  // the partials kernel may still be running: wait for its grid to finish
-  asm volatile("griddepcontrol.wait;" ::: "memory");
 
+  // Everything that does not depend on the partials is done before the wait: the row's
+  // sequence, its chunk range (from cu_seqlens, an input) and the length check.
   const int64_t n_rows = (int64_t)p.B * p.T * p.Hq;
   const int64_t row = (int64_t)blockIdx.x * kMergeRows + warp;
-  uint32_t err = 0u;
-  if (row < n_rows) {
+  const bool has_row = row < n_rows;
+  int n = 0, cbase = 0, rl = 0;
+  bool lengths_ok = false;
+  if (has_row) {
     const int tok = (int)(row / p.Hq), h = (int)(row % p.Hq);
     const int b = tok / p.T, i = tok % p.T;
     const int kh = h / p.g, j = h % p.g;
-    int first = 0, n = 0, total = 0;
+    int first = 0, total = 0;
     sequence_chunks(p, a.cu, b, &first, &n, &total);
     const int32_t L = a.cu[b + 1] - a.cu[b];
     // the device lengths must give the chunk grid the host planned (else some keys were
     // never attended): same chunk count, and a uniform plan long enough for this L
-    const bool lengths_ok = L >= 0 && total == p.n_chunks &&
-                            (p.uniform_n < 0 || (int64_t)prefix_blocks(L) + 1 <= (int64_t)p.uniform_n * p.C);
+    lengths_ok = L >= 0 && total == p.n_chunks &&
+                 (p.uniform_n < 0 || (int64_t)prefix_blocks(L) + 1 <= (int64_t)p.uniform_n * p.C);
+    int32_t u, r;
+    unit_row(p, i, j, &u, &r);
+    rl = r;
+    cbase = first + (kh * p.rg + u) * n;
+  }
+  // the partials kernel may still be running: wait for its grid to finish
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  uint32_t err = 0u;
+  if (has_row) {
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
     float M = -INFINITY, Lsum = 0.f;  // running max of the lse and sum of weights 2^(l - M)
     if (lengths_ok) {
-      int32_t u, rl;
-      unit_row(p, i, j, &u, &rl);
-      const int cbase = first + (kh * p.rg + u) * n;
       for (int x0 = 0; x0 < n; x0 += kPrefetch) {
         const int nx = min(kPrefetch, n - x0);
         // every lane one chunk's lse and status; up to kPrefetch chunk outputs in flight
