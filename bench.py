@@ -280,6 +280,41 @@ def run_ours(args):
         if rc:
             raise binding.LSError(rc, "ls_verify_attn")
 
+    if args.paged:
+        # the same keys in a paged cache: every sequence's pages in random physical order
+        ps = args.paged
+        cu = inp.cu_seqlens
+        n_pages = [(int(x) + ps - 1) // ps for x in np.diff(cu)]
+        total = max(1, sum(n_pages))
+        perm = np.random.default_rng(1234).permutation(total)
+        max_pages = max(1, max(n_pages))
+        table = np.zeros((w.batch, max_pages), dtype=np.int32)
+        src_rows = np.zeros(total * ps, dtype=np.int64)   # packed row of every paged row
+        valid = np.zeros(total * ps, dtype=bool)
+        nxt = 0
+        for b in range(w.batch):
+            for i in range(n_pages[b]):
+                phys = int(perm[nxt])
+                nxt += 1
+                table[b, i] = phys
+                k0, k1 = cu[b] + i * ps, min(cu[b] + (i + 1) * ps, cu[b + 1])
+                src_rows[phys * ps: phys * ps + (k1 - k0)] = np.arange(k0, k1)
+                valid[phys * ps: phys * ps + (k1 - k0)] = True
+        kp = np.where(valid[:, None, None], inp.k_cache[src_rows], 0).astype(np.uint16)
+        vp = np.where(valid[:, None, None], inp.v_cache[src_rows], 0).astype(np.uint16)
+        d_pages = dict(k=bf(kp), v=bf(vp), table=torch.from_numpy(table).to(dev))
+        pg = binding.PagedKV(ps, max_pages, total, d_pages["table"].data_ptr())
+
+        def full_call():  # noqa: F811
+            rc = binding.call_paged_raw(ptr["q"], d_pages["k"].data_ptr(), d_pages["v"].data_ptr(), pg,
+                                        ptr["k_tree"], ptr["v_tree"], ptr["parent"], ptr["cu"], out.data_ptr(),
+                                        lse.data_ptr(), dims, ws, wsb, sp)
+            if rc:
+                raise binding.LSError(rc, "ls_verify_attn_paged")
+
+        partials = full_call  # noqa: F811  (the paged call has no separate partials stage)
+        args.no_e2e = True
+
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
@@ -392,14 +427,17 @@ def run_ours(args):
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16, random draft trees)",
-            "config": config_of(inp, "flushed before every step (write of 2x L2), outside the timed events; "
+            "config": dict(config_of(inp, "flushed before every step (write of 2x L2), outside the timed events; "
                                     "the step is fully queued before its first event"),
+                           **({"kv_layout": f"paged: {args.paged} keys per page, pages in random order"}
+                              if args.paged else {})),
             "kv_hbm_gbs": fig["kv_bytes"] / step_s / 1e9,
             "roofline_step": {"roofline_us": roof_step_s * 1e6, "frac": roof_step_s / step_s,
                               "bytes": fig["step_bytes"], "flops": fig["step_flops"]},
             "roofline": roof, "gpu_launches": 2 * K, "plan": op.plan,
-            "kernel_timing": "partials kernel timed in K further partials-only launches after the K "
-                             "steps, same L2 flush and queueing",
+            "kernel_timing": ("paged call: the roofline figure times the whole call" if args.paged else
+                              "partials kernel timed in K further partials-only launches after the K "
+                              "steps, same L2 flush and queueing"),
             "clocks": sampler.summary(), "e2e": e2e}
     if world == 1 and not args.no_cpu_baseline:
         us, n, dt, cores = time_oracle(inp, target_s=args.cpu_seconds)
@@ -417,6 +455,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE.name, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--paged", type=int, default=0,
+                    help="time ls_verify_attn_paged with pages of this many keys (no e2e figure)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--spin-us", type=float, default=150.0,

@@ -140,6 +140,45 @@ LS_API int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* l
                                   void* stream);
 
 /*
+ * A paged K/V cache. The LongSpec pages keep each sequence's cache contiguous and have no
+ * counterpart; this is the block-table layout of PagedAttention ("Efficient Memory
+ * Management for Large Language Model Serving with PagedAttention", which the mlsanity
+ * page of LongSpec lists under "Builds on"), the layout serving engines use. The keys
+ * of sequence b are still L_b = cu_seqlens[b+1] - cu_seqlens[b] long, but key k of the
+ * sequence lives in row (page_table[b * max_pages_per_seq + k / page_size] * page_size
+ * + k % page_size) of
+ *   k_pages    bf16 [num_pages * page_size, H_kv, d]   (16-byte aligned)
+ *   v_pages    bf16 [num_pages * page_size, H_kv, d]
+ * cu_seqlens then gives only the lengths (its offsets are not used to address the cache).
+ *
+ *   page_size          16, 32, 64, or a multiple of 128 up to 2^20; else LS_ERR_UNSUPPORTED
+ *   max_pages_per_seq  columns of page_table, >= ceil(L_b / page_size) for every planned L_b
+ *   num_pages          pages in k_pages / v_pages; num_pages * page_size < 2^31
+ *   page_table         device int32 [batch, max_pages_per_seq]; an entry outside
+ *                      [0, num_pages) is not an error: the kernel then reads zeros or
+ *                      another page (never memory outside the cache), so the result is
+ *                      unspecified but no fault occurs. Entries past a sequence's last
+ *                      page are not read.
+ */
+typedef struct {
+  int32_t page_size;
+  int32_t max_pages_per_seq;
+  int64_t num_pages;
+  const int32_t* page_table;
+} ls_paged_kv;
+
+/*
+ * ls_verify_attn over a paged K/V cache: the same computation, arguments and errors as
+ * ls_verify_attn, with k_cache / v_cache replaced by the pages and their table. The same
+ * workspace size (ls_verify_attn_workspace_size) applies.
+ */
+LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const ls_paged_kv* paged, const void* k_tree, const void* v_tree,
+                                const int32_t* tree_parent, const int32_t* cu_seqlens, void* out,
+                                float* lse, const ls_verify_dims* dims, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * ls_verify_attn without a workspace argument, for callers that cannot allocate device
  * memory (the LongSpec pages have no counterpart: this is an interface convenience).
  *

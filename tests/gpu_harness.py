@@ -63,20 +63,24 @@ def run_gpu(inp, host_lengths=True, scale=0.0, dev=None, op=None):
 
 def sample_rows(inp, n_random=48, seed=0):
     """Rows r = (b*T+i)*H_q + h covering the first/last node and head of every sequence,
-    the first and last row of every 256-row group of every kv head, plus random rows."""
+    the first and last row of every unit (floor(256/g) whole nodes) of every kv head,
+    both ends of every 128-row query tile inside a unit, plus random rows."""
     w = inp.workload
     B, T, Hq, Hkv = w.batch, w.tree_size, w.num_q_heads, w.num_kv_heads
     g = Hq // Hkv
+    tpu = 256 // g
     rows = set()
     for b in range(B):
         for i in (0, T - 1):
             for h in (0, Hq - 1):
                 rows.add((b * T + i) * Hq + h)
         for kh in range(Hkv):
-            for r_local in range(0, T * g, 256):
-                for rr in (r_local, min(r_local + 255, T * g - 1)):
-                    i, j = divmod(rr, g)
-                    rows.add((b * T + i) * Hq + kh * g + j)
+            for n0 in range(0, T, tpu):
+                n_rows = min(tpu, T - n0) * g
+                for rr in (0, 127, 128, n_rows - 1):
+                    if rr < n_rows:
+                        i, j = divmod(rr, g)
+                        rows.add((b * T + n0 + i) * Hq + kh * g + j)
     rng = np.random.default_rng(seed)
     rows.update(int(x) for x in rng.integers(0, B * T * Hq, size=n_random))
     return np.array(sorted(rows), dtype=np.int64)

@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3:
                 4: "LS_ERR_CUDA", 5: "LS_ERR_BAD_TREE", 6: "LS_ERR_TIMEOUT", 7: "LS_ERR_LENGTHS"}
 EXPORTED = ("ls_verify_attn", "ls_verify_attn_partials", "ls_verify_attn_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
-            "ls_verify_attn_plan", "ls_verify_attn_static")
+            "ls_verify_attn_plan", "ls_verify_attn_static", "ls_verify_attn_paged")
 
 
 class LSError(RuntimeError):
@@ -34,6 +34,11 @@ class LSError(RuntimeError):
         except Exception:
             pass
         super().__init__(f"{what}: {msg}" if what else msg)
+
+
+class PagedKV(ctypes.Structure):
+    _fields_ = [("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int64), ("page_table", ctypes.c_void_p)]
 
 
 class Dims(ctypes.Structure):
@@ -63,6 +68,9 @@ def load_library(path: str = LIB_PATH):
     lib.ls_verify_attn_partials.restype = ctypes.c_int
     lib.ls_verify_attn_combine.argtypes = [P, P, P, D, P, ctypes.c_size_t, P]
     lib.ls_verify_attn_combine.restype = ctypes.c_int
+    lib.ls_verify_attn_paged.argtypes = [P, P, P, ctypes.POINTER(PagedKV), P, P, P, P, P, P, D, P,
+                                         ctypes.c_size_t, P]
+    lib.ls_verify_attn_paged.restype = ctypes.c_int
     lib.ls_verify_attn_static.argtypes = [P, P, P, P, P, P, P, P, P, D, P]
     lib.ls_verify_attn_static.restype = ctypes.c_int
     lib.ls_verify_attn_workspace_size.argtypes = [D]
@@ -121,6 +129,14 @@ def call_static_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, out
     callers that cannot allocate device memory; returns the status code."""
     return int(load_library().ls_verify_attn_static(q, k_cache, v_cache, k_tree, v_tree, parent,
                                                     cu_seqlens, out, lse, ctypes.byref(dims), stream))
+
+
+def call_paged_raw(q, k_pages, v_pages, paged: PagedKV, k_tree, v_tree, parent, cu_seqlens, out, lse,
+                   dims: Dims, workspace, workspace_bytes: int, stream) -> int:
+    """ls_verify_attn_paged on raw device addresses (ints); returns the status code."""
+    return int(load_library().ls_verify_attn_paged(q, k_pages, v_pages, ctypes.byref(paged), k_tree, v_tree,
+                                                   parent, cu_seqlens, out, lse, ctypes.byref(dims), workspace,
+                                                   workspace_bytes, stream))
 
 
 def call_partials_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, dims: Dims, workspace,

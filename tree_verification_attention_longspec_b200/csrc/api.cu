@@ -2,6 +2,7 @@
 // Declared and documented in include/ls_verify_attn.h.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <vector>
@@ -152,9 +153,14 @@ int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* partials_ctas, int3
   return LS_OK;
 }
 
-int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree,
-                            const void* v_tree, const int32_t* tree_parent, const int32_t* cu_seqlens,
-                            const ls_verify_dims* dims, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The partials stage for a packed (pg == nullptr) or paged K/V cache; arguments checked.
+int run_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree, const void* v_tree,
+                 const int32_t* tree_parent, const int32_t* cu_seqlens, const ls_verify_dims* dims,
+                 const ls_paged_kv* pg, void* workspace, size_t workspace_bytes, void* stream) {
   Plan p;
   int rc = make_plan(dims, &p);
   if (rc != LS_OK) return rc;
@@ -163,9 +169,28 @@ int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_ca
     if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
   if (tree_parent == nullptr || cu_seqlens == nullptr || !aligned4(tree_parent) || !aligned4(cu_seqlens))
     return LS_ERR_INVALID_ARG;
+  const bool any_prefix =
+      dims->cu_seqlens_host ? dims->cu_seqlens_host[dims->batch] > 0 : dims->max_prefix_len > 0;
+  int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
+                                          : (int64_t)dims->batch * dims->max_prefix_len;
+  if (pg != nullptr) {
+    // pages of 16, 32 or 64 keys, or a multiple of 128 (a 128-key block never straddles
+    // two pages then); enough table columns for the longest planned sequence
+    const int32_t ps = pg->page_size;
+    if (!(ps == 16 || ps == 32 || ps == 64 || (ps >= 128 && ps % 128 == 0 && ps <= (1 << 20))))
+      return LS_ERR_UNSUPPORTED;
+    if (pg->page_table == nullptr || !aligned4(pg->page_table) || pg->max_pages_per_seq < 1 || pg->num_pages < 1)
+      return LS_ERR_INVALID_ARG;
+    int64_t max_len = dims->max_prefix_len;
+    if (dims->cu_seqlens_host)
+      for (int b = 0; b < dims->batch; ++b)
+        max_len = std::max<int64_t>(max_len, dims->cu_seqlens_host[b + 1] - dims->cu_seqlens_host[b]);
+    if ((max_len + ps - 1) / ps > pg->max_pages_per_seq) return LS_ERR_INVALID_ARG;
+    if (pg->num_pages * (int64_t)ps >= (int64_t)1 << 31) return LS_ERR_UNSUPPORTED;  // rows stay int32
+    kv_rows = pg->num_pages * (int64_t)ps;
+  }
   if (k_cache == nullptr || v_cache == nullptr || !aligned16(k_cache) || !aligned16(v_cache)) {
     // a call without prefix keys may pass null caches
-    const bool any_prefix = dims->cu_seqlens_host ? dims->cu_seqlens_host[dims->batch] > 0 : dims->max_prefix_len > 0;
     if (any_prefix || (k_cache != nullptr && !aligned16(k_cache)) || (v_cache != nullptr && !aligned16(v_cache)))
       return LS_ERR_INVALID_ARG;
   }
@@ -182,18 +207,30 @@ int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_ca
   pa.v_tree = static_cast<const uint16_t*>(v_tree);
   pa.parent = tree_parent;
   pa.cu = cu_seqlens;
+  pa.page_table = pg ? pg->page_table : nullptr;
+  pa.page_size = pg ? pg->page_size : 0;
+  pa.max_pages = pg ? pg->max_pages_per_seq : 0;
   pa.o_part = reinterpret_cast<float*>(ws + lay.o_part);
   pa.lse_part = reinterpret_cast<float*>(ws + lay.lse_part);
   pa.chunk_status = reinterpret_cast<uint32_t*>(ws + lay.chunk_status);
   pa.p = p;
   // rows of the K/V tensors that the TMA descriptors may address (an upper bound is
-  // enough: no block is ever read past its sequence's end)
-  int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
-                                          : (int64_t)dims->batch * dims->max_prefix_len;
+  // enough: no block is ever read past the tensor)
   if (k_cache == nullptr) kv_rows = (int64_t)p.B * p.T;
   const cudaError_t e = ls::launch_partials(pa, kv_rows, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree,
+                            const void* v_tree, const int32_t* tree_parent, const int32_t* cu_seqlens,
+                            const ls_verify_dims* dims, void* workspace, size_t workspace_bytes, void* stream) {
+  return run_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, nullptr, workspace,
+                      workspace_bytes, stream);
 }
 
 int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims,
@@ -231,6 +268,21 @@ int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache, cons
   if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
   rc = ls_verify_attn_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, workspace,
                                workspace_bytes, stream);
+  if (rc != LS_OK) return rc;
+  return ls_verify_attn_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream);
+}
+
+int ls_verify_attn_paged(const void* q, const void* k_pages, const void* v_pages, const ls_paged_kv* paged,
+                         const void* k_tree, const void* v_tree, const int32_t* tree_parent,
+                         const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(dims, &p);
+  if (rc != LS_OK) return rc;
+  if (paged == nullptr) return LS_ERR_INVALID_ARG;
+  if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
+  rc = run_partials(q, k_pages, v_pages, k_tree, v_tree, tree_parent, cu_seqlens, dims, paged, workspace,
+                    workspace_bytes, stream);
   if (rc != LS_OK) return rc;
   return ls_verify_attn_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream);
 }

@@ -19,6 +19,11 @@ struct PartialsArgs {
   const uint16_t* v_tree;
   const int32_t* parent;
   const int32_t* cu;
+  // paged K/V cache: page_table[b * max_pages + i] is the physical page of keys
+  // [i * page_size, (i + 1) * page_size) of sequence b; nullptr = keys packed by cu
+  const int32_t* page_table;
+  int32_t page_size;
+  int32_t max_pages;
   float* o_part;
   float* lse_part;
   uint32_t* chunk_status;
@@ -56,6 +61,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Launchers (defined in the kernel files, called by the host API).
 namespace ls {
-cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream);
+cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream);  // kv_rows: rows of the K/V tensors
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 }  // namespace ls

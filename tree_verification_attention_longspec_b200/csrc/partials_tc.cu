@@ -204,7 +204,13 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   if (!c.valid) return;  // more CTAs than the device lengths need: the combine reports it
   const int n_keys = c.key_end - c.key_begin;
   const int nb = (n_keys + kBlockN - 1) / kBlockN;  // prefix blocks
-  const int tail_shift = nb * kBlockN - n_keys;      // masked leading columns of the last one
+  // The last prefix block of a packed cache is loaded as the box that ends at the
+  // sequence end (its leading tail_shift columns are earlier keys, masked); in a paged
+  // cache it is loaded from its aligned start, page by page, and its columns from
+  // tail_end on lie past the sequence end (masked).
+  const bool paged = a.page_table != nullptr;
+  const int tail_shift = paged ? 0 : nb * kBlockN - n_keys;
+  const int tail_end = paged ? n_keys - (nb - 1) * kBlockN : kBlockN;
   const bool has_tree = c.has_tree;
   const int nbt = nb + (has_tree ? 1 : 0);  // blocks, the tree block (block nb) last
   const int tok0 = c.rgi * p.tpu;                    // first tree node of the unit
@@ -258,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     // ------------------------------------------------------------------ TMA producer
     // Ring order = consumption order: K(0), V(0), K(1), V(1), ...
     if (lane == 0) {
+      const int seq_len = a.cu[c.b + 1] - a.cu[c.b];
       // Q first: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows
       // past the batch's last node read as zeros)
       mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
@@ -274,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         int row = c.seq_offset + c.key_begin + j * kBlockN;
         if (j == nb - 1) row -= tail_shift;  // the box ends at the sequence end
         if (tree) row = c.b * p.T;
+        const bool pieces = paged && !tree;  // the block's rows come page by page
         for (int kv = 0; kv < 2; ++kv) {
           if (!mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs)) {
             ok = false;
@@ -282,9 +290,28 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           mbar_arrive_expect_tx(&bars->full[slot], C::kTileBytes);
           uint8_t* dst = smem + C::kSlotOff + slot * C::kTileBytes;
           const CUtensorMap* map = tree ? (kv ? &P.tmap_vt : &P.tmap_kt) : (kv ? &P.tmap_v : &P.tmap_k);
+          if (!pieces) {
 #pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
+          } else {
+            // boxes of bh rows (the page, or 128 rows of a larger page); pieces past the
+            // sequence end read its last page (masked). A page-table entry is only a TMA
+            // coordinate, so a bad one reads zeros or another page, never outside the cache.
+            const int bh = a.page_size < kBlockN ? a.page_size : kBlockN;
+            const int n_pages = (seq_len + a.page_size - 1) / a.page_size;
+            for (int pc = 0; pc < kBlockN / bh; ++pc) {
+              const int key = c.key_begin + j * kBlockN + pc * bh;
+              int lp = key / a.page_size;
+              if (lp >= n_pages) lp = n_pages - 1;
+              if (lp >= a.max_pages) lp = a.max_pages - 1;
+              const int prow = a.page_table[(size_t)c.b * a.max_pages + lp] * a.page_size + key % a.page_size;
+#pragma unroll
+              for (int pn = 0; pn < C::kPanels; ++pn)
+                tma_load_3d(dst + pn * C::kPanelBytes + pc * bh * 128, map, &bars->full[slot], pn * 64, c.kh,
+                            prow);
+            }
+          }
           ++issued;
           if (++slot == C::kSlots) {
             slot = 0;
@@ -437,7 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], j & 1, abort, kTimeoutNs));
         if (!ok) break;
         tc_fence_after_sync();
-        const int shift = j == nb - 1 ? tail_shift : 0;  // masked leading columns
+        const int shift = j == nb - 1 ? tail_shift : 0;    // masked leading columns
+        const int lim = j == nb - 1 ? tail_end : kBlockN;  // columns from here on are masked
         const bool tree_blk = j == nb;                      // keys = the sequence's tree nodes
         if (tree_blk && mask_tree_scores(bars->parent, tS, has_row ? node : -1)) bars->tree_err = 1u;
         // All 128 scores for the row maximum; the scores of keys 0..63 stay in registers
@@ -455,11 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             lo[e] = __uint_as_float(r[e >> 5][e & 31]);
             hi[e] = __uint_as_float(r[2 + (e >> 5)][e & 31]);
           }
-          if (shift > 0) {  // the sequence's last block: these columns are earlier keys
+          if (shift > 0 || lim < kBlockN) {  // the sequence's last prefix block
 #pragma unroll
             for (int e = 0; e < kHalf; ++e) {
-              if (e < shift) lo[e] = -INFINITY;
-              if (e + kHalf < shift) hi[e] = -INFINITY;
+              if (e < shift || e >= lim) lo[e] = -INFINITY;
+              if (e + kHalf < shift || e + kHalf >= lim) hi[e] = -INFINITY;
             }
           }
           float m0 = fmaxf(lo[0], hi[0]), m1 = fmaxf(lo[1], hi[1]);
@@ -476,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         const bool raise = mx > m + kRescaleThreshold;
         const bool any_raise = __any_sync(0xffffffffu, raise);
         // masked columns (-inf) and the rare blocks that raise m take the MUFU-only path
-        const bool mufu_only = EMU == 0 || shift > 0 || tree_blk || any_raise;
+        const bool mufu_only = EMU == 0 || shift > 0 || lim < kBlockN || tree_blk || any_raise;
         const float m_new = raise ? mx : m;
         // a row that has seen no visible key yet (a padding row of a tree-only chunk)
         // keeps m = -inf; its P is 0 against any finite reference
@@ -518,10 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < kHalf; ++e) hi[e] = __uint_as_float(r[e >> 5][e & 31]);
-          if (shift > kHalf) {
+          if (shift > kHalf || lim < kBlockN) {
 #pragma unroll
             for (int e = 0; e < kHalf; ++e)
-              if (e + kHalf < shift) hi[e] = -INFINITY;
+              if (e + kHalf < shift || e + kHalf >= lim) hi[e] = -INFINITY;
           }
         }
         {
@@ -609,12 +637,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // K or V cache viewed as [rows][H_kv][D] bf16; boxes of 128 rows x 64 elements of one head.
-bool make_kv_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t rows) {
+bool make_kv_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t rows, int box_rows = 128) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -642,8 +670,10 @@ cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream
   TcParams P;
   P.a = a;
   const int64_t tree_rows = (int64_t)a.p.B * a.p.T;
-  if (!make_q_map(&P.tmap_q, a.q, D, a.p) || !make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows) ||
-      !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows) ||
+  // a paged cache is read in boxes of one page (at most 128 rows)
+  const int box_rows = a.page_table != nullptr && a.page_size < kBlockN ? a.page_size : kBlockN;
+  if (!make_q_map(&P.tmap_q, a.q, D, a.p) || !make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows, box_rows) ||
+      !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows, box_rows) ||
       !make_kv_map(&P.tmap_kt, a.k_tree, D, a.p.Hkv, tree_rows) ||
       !make_kv_map(&P.tmap_vt, a.v_tree, D, a.p.Hkv, tree_rows))
     return cudaErrorInvalidValue;
