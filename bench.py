@@ -14,6 +14,7 @@ is the max over ranks. Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -48,10 +49,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_figures(inp):
+def workload_figures(inp, cross=False):
     w = inp.workload
     L = inp.prefix_lengths
     total_L = int(L.sum())
+    if cross:
+        # prefix-only attention: 4*d flops per (query row, prefix key); bytes: the prefix
+        # K/V, the queries, out and lse
+        rows = w.batch * w.tree_size * w.num_q_heads
+        kv_bytes = 4 * total_L * w.num_kv_heads * w.head_dim
+        flops = 4 * w.head_dim * w.tree_size * w.num_q_heads * total_L
+        step_bytes = kv_bytes + 4 * rows * w.head_dim + 4 * rows
+        return dict(total_L=total_L, step_bytes=step_bytes, step_flops=flops, partials_flops=flops,
+                    partials_bytes=kv_bytes + 2 * rows * w.head_dim, kv_bytes=kv_bytes, rows=rows)
     step_bytes = algorithmic_bytes(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.tree_size,
                                    total_L)
     step_flops = algorithmic_flops(w.num_q_heads, w.head_dim, w.tree_size, L)
@@ -248,8 +258,11 @@ def run_ours(args):
     binding.load_library()
 
     w = WORKLOADS[args.workload]
+    if args.cross:
+        # the draft's cross-attention: args.cross queries per sequence over the same cache
+        w = dataclasses.replace(w, name=f"{w.name}_cross{args.cross}", tree_size=args.cross, tree="chain")
     inp = make_inputs(w, seed=rank)   # independent problem per rank
-    fig = workload_figures(inp)
+    fig = workload_figures(inp, cross=bool(args.cross))
 
     def bf(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -279,6 +292,22 @@ def run_ours(args):
                               ptr["parent"], ptr["cu"], out.data_ptr(), lse.data_ptr(), dims, ws, wsb, sp)
         if rc:
             raise binding.LSError(rc, "ls_verify_attn")
+
+    def check_status():
+        return binding.check(dims, ws_x.data_ptr(), sp) if args.cross else op.check()
+
+    if args.cross:
+        wsb_x = binding.cross_workspace_size(dims)
+        ws_x = torch.empty(wsb_x, dtype=torch.uint8, device=dev)
+
+        def full_call():  # noqa: F811
+            rc = binding.call_cross_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["cu"], out.data_ptr(),
+                                        lse.data_ptr(), dims, ws_x.data_ptr(), wsb_x, sp)
+            if rc:
+                raise binding.LSError(rc, "ls_cross_attn")
+
+        partials = full_call  # noqa: F811  (timed as one call)
+        args.no_e2e = True
 
     if args.paged:
         # the same keys in a paged cache: every sequence's pages in random physical order
@@ -324,7 +353,7 @@ def run_ours(args):
         flush.zero_()
         partials()
     torch.cuda.synchronize(dev)
-    st = op.check()
+    st = check_status()
     if st != 0:
         raise binding.LSError(st, "device status after warm-up")
 
@@ -363,7 +392,7 @@ def run_ours(args):
     ms_per_step = float(statistics.mean(step_ms))
     partials_avg_ms = float(statistics.mean(partials_ms))
     ms_per_step, partials_avg_ms = max_over_ranks([ms_per_step, partials_avg_ms], device=dev)
-    st = op.check()
+    st = check_status()
     if st != 0:
         raise binding.LSError(st, "device status after timing")
 
@@ -430,12 +459,15 @@ def run_ours(args):
             "config": dict(config_of(inp, "flushed before every step (write of 2x L2), outside the timed events; "
                                     "the step is fully queued before its first event"),
                            **({"kv_layout": f"paged: {args.paged} keys per page, pages in random order"}
-                              if args.paged else {})),
+                              if args.paged else {}),
+                           **({"attention": f"prefix-only (ls_cross_attn), {args.cross} queries per sequence"}
+                              if args.cross else {})),
             "kv_hbm_gbs": fig["kv_bytes"] / step_s / 1e9,
             "roofline_step": {"roofline_us": roof_step_s * 1e6, "frac": roof_step_s / step_s,
                               "bytes": fig["step_bytes"], "flops": fig["step_flops"]},
             "roofline": roof, "gpu_launches": 2 * K, "plan": op.plan,
-            "kernel_timing": ("paged call: the roofline figure times the whole call" if args.paged else
+            "kernel_timing": ("paged or cross-attention call: the roofline figure times the whole call"
+                              if (args.paged or args.cross) else
                               "partials kernel timed in K further partials-only launches after the K "
                               "steps, same L2 flush and queueing"),
             "clocks": sampler.summary(), "e2e": e2e}
@@ -455,6 +487,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE.name, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cross", type=int, default=0,
+                    help="time ls_cross_attn (prefix-only attention) with this many queries per sequence")
     ap.add_argument("--paged", type=int, default=0,
                     help="time ls_verify_attn_paged with pages of this many keys (no e2e figure)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -179,6 +179,28 @@ LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* 
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * Prefix-only attention: the draft model's cross-attention over the target model's KV
+ * cache (LongSpec, gist.science summary, section 2A, "Cross-Attention mit geteiltem
+ * KV-Cache": the draft reads the target's cache directly, so long contexts cost it no
+ * cache of its own). Every query of sequence b attends to all L_b keys of its sequence
+ * in k_cache / v_cache with no mask, and to nothing else: there are no tree keys.
+ *
+ *   q          bf16 [B*T, H_q, d]   T = dims->tree_size queries per sequence (1..128)
+ *   k_cache    bf16 [sum_b L_b, H_kv, d], v_cache likewise, packed by cu_seqlens (may be
+ *              NULL when every L_b is 0)
+ *   out, lse   as for ls_verify_attn; a sequence with L_b = 0 gets out = 0, lse = -inf
+ *   workspace  at least ls_cross_attn_workspace_size(dims) bytes (it differs from
+ *              ls_verify_attn_workspace_size: the key lists have no tree block)
+ * Errors as for ls_verify_attn; ls_verify_attn_check reads its device status.
+ * (The draft's sliding-window self-attention is ls_verify_attn itself: the window's
+ * cache as the prefix and the new draft tokens as a chain tree.)
+ */
+LS_API size_t ls_cross_attn_workspace_size(const ls_verify_dims* dims);
+LS_API int ls_cross_attn(const void* q, const void* k_cache, const void* v_cache, const int32_t* cu_seqlens,
+                         void* out, float* lse, const ls_verify_dims* dims, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
  * ls_verify_attn without a workspace argument, for callers that cannot allocate device
  * memory (the LongSpec pages have no counterpart: this is an interface convenience).
  *

@@ -2,7 +2,8 @@
 // covered by exactly one chunk, where the key blocks of a sequence are its 128-key
 // prefix blocks followed by its tree block; chunk ids are dense, and the per-sequence
 // chunk ranges that the combine kernel uses agree with locate_chunk.
-// Usage: plan_check B Hq Hkv T C uniform_n L_0 ... L_{B-1}   (exit 0 = pass)
+// Usage: plan_check B Hq Hkv T C uniform_n L_0 ... L_{B-1}   (exit 0 = pass); with
+// PLAN_CHECK_NO_TREE set, the key lists hold the prefix blocks only.
 #include <cstdio>
 #include <cstdlib>
 #include <map>
@@ -25,6 +26,7 @@ int main(int argc, char** argv) {
   p.rows = p.T * p.g;
   p.tpu = ls::kUnitRows / p.g;
   p.rg = ls::ceil_div(p.T, p.tpu);
+  p.with_tree = getenv("PLAN_CHECK_NO_TREE") ? 0 : 1;  // prefix-only plans (cross-attention)
   if (argc != 7 + p.B) return 2;
   std::vector<int32_t> cu(p.B + 1, 0);
   for (int b = 0; b < p.B; ++b) cu[b + 1] = cu[b] + atoi(argv[7 + b]);
@@ -53,7 +55,7 @@ int main(int argc, char** argv) {
     const int L = cu[b + 1] - cu[b];
     for (int kh = 0; kh < p.Hkv; ++kh)
       for (int r = 0; r < p.rg; ++r)
-        for (int k = 0; k <= ls::prefix_blocks(L); ++k) {
+        for (int k = 0; k < ls::prefix_blocks(L) + p.with_tree; ++k) {
           auto it = seen.find(std::make_tuple(b, kh, r, k));
           if (it == seen.end() || it->second != 1) {
             printf("block (%d,%d,%d,%d) covered %d times\n", b, kh, r, k,

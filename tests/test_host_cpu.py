@@ -39,6 +39,19 @@ def test_chunk_plan_covers_every_block_once(plan_check, B, Hq, Hkv, T, C, unifor
     assert r.returncode == 0, r.stdout + r.stderr
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,T,C,uniform,lengths", [
+    (1, 28, 4, 1, 14, -1, [65536]),
+    (3, 8, 2, 4, 3, -1, [0, 129, 1000]),
+    (2, 8, 8, 1, 5, 2, [640, 7]),
+])
+def test_prefix_only_plan_covers_every_prefix_block_once(plan_check, B, Hq, Hkv, T, C, uniform, lengths):
+    # cross-attention plans: the key lists hold the prefix blocks only (no tree block)
+    env = dict(os.environ, PLAN_CHECK_NO_TREE="1")
+    r = subprocess.run([plan_check, str(B), str(Hq), str(Hkv), str(T), str(C), str(uniform),
+                        *map(str, lengths)], capture_output=True, text=True, env=env)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_plan_check_catches_an_uncovered_tree_block(plan_check):
     # uniform plan of 3 chunks of 5 blocks: 1920 keys need 15 prefix blocks and the tree
     # block, 16 in all, so the tree block of that sequence is left out

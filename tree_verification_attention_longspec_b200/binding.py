@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3:
                 4: "LS_ERR_CUDA", 5: "LS_ERR_BAD_TREE", 6: "LS_ERR_TIMEOUT", 7: "LS_ERR_LENGTHS"}
 EXPORTED = ("ls_verify_attn", "ls_verify_attn_partials", "ls_verify_attn_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
-            "ls_verify_attn_plan", "ls_verify_attn_static", "ls_verify_attn_paged")
+            "ls_verify_attn_plan", "ls_verify_attn_static", "ls_verify_attn_paged", "ls_cross_attn",
+            "ls_cross_attn_workspace_size")
 
 
 class LSError(RuntimeError):
@@ -71,6 +72,10 @@ def load_library(path: str = LIB_PATH):
     lib.ls_verify_attn_paged.argtypes = [P, P, P, ctypes.POINTER(PagedKV), P, P, P, P, P, P, D, P,
                                          ctypes.c_size_t, P]
     lib.ls_verify_attn_paged.restype = ctypes.c_int
+    lib.ls_cross_attn.argtypes = [P, P, P, P, P, P, D, P, ctypes.c_size_t, P]
+    lib.ls_cross_attn.restype = ctypes.c_int
+    lib.ls_cross_attn_workspace_size.argtypes = [D]
+    lib.ls_cross_attn_workspace_size.restype = ctypes.c_size_t
     lib.ls_verify_attn_static.argtypes = [P, P, P, P, P, P, P, P, P, D, P]
     lib.ls_verify_attn_static.restype = ctypes.c_int
     lib.ls_verify_attn_workspace_size.argtypes = [D]
@@ -137,6 +142,17 @@ def call_paged_raw(q, k_pages, v_pages, paged: PagedKV, k_tree, v_tree, parent, 
     return int(load_library().ls_verify_attn_paged(q, k_pages, v_pages, ctypes.byref(paged), k_tree, v_tree,
                                                    parent, cu_seqlens, out, lse, ctypes.byref(dims), workspace,
                                                    workspace_bytes, stream))
+
+
+def cross_workspace_size(dims: Dims) -> int:
+    return int(load_library().ls_cross_attn_workspace_size(ctypes.byref(dims)))
+
+
+def call_cross_raw(q, k_cache, v_cache, cu_seqlens, out, lse, dims: Dims, workspace, workspace_bytes: int,
+                   stream) -> int:
+    """ls_cross_attn (prefix-only attention) on raw device addresses; returns the status code."""
+    return int(load_library().ls_cross_attn(q, k_cache, v_cache, cu_seqlens, out, lse, ctypes.byref(dims),
+                                            workspace, workspace_bytes, stream))
 
 
 def call_partials_raw(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, dims: Dims, workspace,

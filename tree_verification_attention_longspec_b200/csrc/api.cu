@@ -63,7 +63,7 @@ int check_dims(const ls_verify_dims* d) {
 // the partials kernel: waves of `slots` CTAs, each wave as long as its longest chunk
 // plus a fixed per-chunk cost for loading Q and writing the partial. A sequence's key
 // list is its prefix blocks plus one tree block.
-int make_plan(const ls_verify_dims* d, Plan* p) {
+int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true) {
   int rc = check_dims(d);
   if (rc != LS_OK) return rc;
   int sms = 0, major = 0;
@@ -91,13 +91,13 @@ int make_plan(const ls_verify_dims* d, Plan* p) {
   for (int b = 0; b < q.B; ++b) {
     const int32_t L = d->cu_seqlens_host ? d->cu_seqlens_host[b + 1] - d->cu_seqlens_host[b]
                                          : d->max_prefix_len;
-    blocks[b] = ls::prefix_blocks(L) + 1;  // prefix blocks and the tree block
+    blocks[b] = ls::prefix_blocks(L) + (with_tree ? 1 : 0);  // prefix blocks and the tree block
     if (blocks[b] > max_blocks) max_blocks = blocks[b];
   }
   const long long units = (long long)q.Hkv * q.rg;
   const long long slots = sms;  // one prefix CTA per SM
   const long long overhead = 2;  // per-chunk cost in blocks (Q load, partial store)
-  int32_t best_C = max_blocks;
+  int32_t best_C = max_blocks > 0 ? max_blocks : 1;
   long long best_cost = -1, best_n = 0;
   for (int32_t C = 1; C <= max_blocks; ++C) {
     long long n = 0;
@@ -111,10 +111,11 @@ int make_plan(const ls_verify_dims* d, Plan* p) {
     }
   }
   q.C = best_C;
+  q.with_tree = with_tree ? 1 : 0;
   if (d->cu_seqlens_host) {
     q.uniform_n = -1;
   } else {
-    q.uniform_n = ls::ceil_div(max_blocks, q.C);
+    q.uniform_n = max_blocks > 0 ? ls::ceil_div(max_blocks, q.C) : 0;
   }
   long long n = 0;
   for (int b = 0; b < q.B; ++b)
@@ -160,15 +161,17 @@ namespace {
 // The partials stage for a packed (pg == nullptr) or paged K/V cache; arguments checked.
 int run_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree, const void* v_tree,
                  const int32_t* tree_parent, const int32_t* cu_seqlens, const ls_verify_dims* dims,
-                 const ls_paged_kv* pg, void* workspace, size_t workspace_bytes, void* stream) {
+                 const ls_paged_kv* pg, void* workspace, size_t workspace_bytes, void* stream,
+                 bool with_tree = true) {
   Plan p;
-  int rc = make_plan(dims, &p);
+  int rc = make_plan(dims, &p, with_tree);
   if (rc != LS_OK) return rc;
-  const void* ptrs16[] = {q, k_tree, v_tree};
-  for (const void* x : ptrs16)
-    if (x == nullptr || !aligned16(x)) return LS_ERR_INVALID_ARG;
-  if (tree_parent == nullptr || cu_seqlens == nullptr || !aligned4(tree_parent) || !aligned4(cu_seqlens))
-    return LS_ERR_INVALID_ARG;
+  if (q == nullptr || !aligned16(q) || cu_seqlens == nullptr || !aligned4(cu_seqlens)) return LS_ERR_INVALID_ARG;
+  if (with_tree) {
+    if (k_tree == nullptr || v_tree == nullptr || !aligned16(k_tree) || !aligned16(v_tree))
+      return LS_ERR_INVALID_ARG;
+    if (tree_parent == nullptr || !aligned4(tree_parent)) return LS_ERR_INVALID_ARG;
+  }
   const bool any_prefix =
       dims->cu_seqlens_host ? dims->cu_seqlens_host[dims->batch] > 0 : dims->max_prefix_len > 0;
   int64_t kv_rows = dims->cu_seqlens_host ? (int64_t)dims->cu_seqlens_host[dims->batch]
@@ -194,17 +197,18 @@ int run_partials(const void* q, const void* k_cache, const void* v_cache, const 
     if (any_prefix || (k_cache != nullptr && !aligned16(k_cache)) || (v_cache != nullptr && !aligned16(v_cache)))
       return LS_ERR_INVALID_ARG;
   }
+  if (!with_tree && p.n_chunks == 0) return LS_OK;  // no key at all: the combine writes the empty result
   const ls::Layout lay = ls::make_layout(p);
   if (!workspace_ok(workspace, workspace_bytes, lay)) return LS_ERR_WORKSPACE;
   char* ws = static_cast<char*>(workspace);
   (void)cudaGetLastError();  // clear a stale, non-sticky error from unrelated work
   ls::PartialsArgs pa;
   pa.q = static_cast<const uint16_t*>(q);
-  // the tensor maps need an address even where no prefix row is ever read
+  // the tensor maps need an address even where no row is ever read through them
   pa.k_cache = static_cast<const uint16_t*>(k_cache ? k_cache : k_tree);
   pa.v_cache = static_cast<const uint16_t*>(v_cache ? v_cache : v_tree);
-  pa.k_tree = static_cast<const uint16_t*>(k_tree);
-  pa.v_tree = static_cast<const uint16_t*>(v_tree);
+  pa.k_tree = static_cast<const uint16_t*>(with_tree ? k_tree : k_cache);
+  pa.v_tree = static_cast<const uint16_t*>(with_tree ? v_tree : v_cache);
   pa.parent = tree_parent;
   pa.cu = cu_seqlens;
   pa.page_table = pg ? pg->page_table : nullptr;
@@ -233,10 +237,14 @@ int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_ca
                       workspace_bytes, stream);
 }
 
-int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims,
-                           void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int run_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims, void* workspace,
+                size_t workspace_bytes, void* stream, bool with_tree) {
   Plan p;
-  int rc = make_plan(dims, &p);
+  int rc = make_plan(dims, &p, with_tree);
   if (rc != LS_OK) return rc;
   if (out == nullptr || !aligned16(out)) return LS_ERR_INVALID_ARG;
   if (cu_seqlens == nullptr || lse == nullptr || !aligned4(cu_seqlens) || !aligned4(lse)) return LS_ERR_INVALID_ARG;
@@ -255,6 +263,33 @@ int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* lse, con
   ca.p = p;
   if (ls::launch_combine(ca, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ls_verify_attn_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, true);
+}
+
+size_t ls_cross_attn_workspace_size(const ls_verify_dims* dims) {
+  Plan p;
+  if (make_plan(dims, &p, false) != LS_OK) return 0;
+  return (size_t)ls::make_layout(p).total;
+}
+
+int ls_cross_attn(const void* q, const void* k_cache, const void* v_cache, const int32_t* cu_seqlens, void* out,
+                  float* lse, const ls_verify_dims* dims, void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(dims, &p, false);
+  if (rc != LS_OK) return rc;
+  if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
+  rc = run_partials(q, k_cache, v_cache, nullptr, nullptr, nullptr, cu_seqlens, dims, nullptr, workspace,
+                    workspace_bytes, stream, false);
+  if (rc != LS_OK) return rc;
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, false);
 }
 
 int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache, const void* k_tree,

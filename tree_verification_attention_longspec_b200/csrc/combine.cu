@@ -45,7 +45,7 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
     // the device lengths must give the chunk grid the host planned (else some keys were
     // never attended): same chunk count, and a uniform plan long enough for this L
     lengths_ok = L >= 0 && total == p.n_chunks &&
-                 (p.uniform_n < 0 || (int64_t)prefix_blocks(L) + 1 <= (int64_t)p.uniform_n * p.C);
+                 (p.uniform_n < 0 || (int64_t)prefix_blocks(L) + p.with_tree <= (int64_t)p.uniform_n * p.C);
     int32_t u, r;
     unit_row(p, i, j, &u, &r);
     rl = r;

@@ -38,6 +38,7 @@ struct Plan {
   int32_t tpu;         // tree nodes per unit: floor(kUnitRows / g)
   int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
   int32_t C;           // 128-key blocks per chunk
+  int32_t with_tree;   // 1: every key list ends with the tree block; 0: prefix keys only
   int32_t uniform_n;   // >= 0: chunks per unit for every sequence; -1: from L_b
   int32_t n_chunks;    // partials-kernel CTAs
   int32_t n_combine;   // combine CTAs = ceil(B * T * Hq / kMergeRows)
@@ -51,10 +52,10 @@ LS_HD int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
 LS_HD int32_t prefix_blocks(int32_t L) { return L > 0 ? ceil_div(L, kBlockN) : 0; }
 
 // chunks of one (sequence, kv head, unit) for a prefix of L keys: its prefix blocks
-// and the tree block, C per chunk
+// and (with_tree) the tree block, C per chunk
 LS_HD int32_t chunks_per_unit(const Plan& p, int32_t L) {
   if (p.uniform_n >= 0) return p.uniform_n;
-  return ceil_div(prefix_blocks(L) + 1, p.C);
+  return ceil_div(prefix_blocks(L) + p.with_tree, p.C);
 }
 
 // Unit and row inside the unit of query row (tree node i, head-in-group j).
@@ -96,7 +97,7 @@ LS_HD ChunkCoord locate_chunk(const Plan& p, const int32_t* cu, int32_t cid) {
       c.key_begin = kb < Lc ? kb : Lc;
       c.key_end = ke < Lc ? ke : Lc;
       const int32_t tree_block = prefix_blocks(Lc);
-      c.has_tree = v0 <= tree_block && tree_block < v1;
+      c.has_tree = p.with_tree && v0 <= tree_block && tree_block < v1;
       c.valid = true;
       return c;
     }
@@ -120,12 +121,13 @@ LS_HD void sequence_chunks(const Plan& p, const int32_t* cu, int32_t b, int32_t*
   *total = base;
 }
 
-// Workspace layout (byte offsets, each 256-aligned).
+// Workspace layout (byte offsets, each 256-aligned). The combine's status words come
+// first, so that their place depends on the output rows alone, not on the chunk plan.
 struct Layout {
-  uint64_t o_part;        // float [n_chunks][kUnitRows][d]   prefix partial out, normalised
-  uint64_t lse_part;      // float [n_chunks][kUnitRows]      prefix partial lse, log2 domain
-  uint64_t chunk_status;  // u32   [n_chunks]
   uint64_t status;        // u32   [n_combine]
+  uint64_t o_part;        // float [n_chunks][kUnitRows][d]   partial out, normalised
+  uint64_t lse_part;      // float [n_chunks][kUnitRows]      partial lse, log2 domain
+  uint64_t chunk_status;  // u32   [n_chunks]
   uint64_t total;
 };
 
@@ -134,14 +136,14 @@ LS_HD uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 LS_HD Layout make_layout(const Plan& p) {
   Layout l{};
   uint64_t off = 0;
+  l.status = off;
+  off = align256(off + (uint64_t)p.n_combine * 4);
   l.o_part = off;
   off = align256(off + (uint64_t)p.n_chunks * kUnitRows * p.d * 4);
   l.lse_part = off;
   off = align256(off + (uint64_t)p.n_chunks * kUnitRows * 4);
   l.chunk_status = off;
   off = align256(off + (uint64_t)p.n_chunks * 4);
-  l.status = off;
-  off = align256(off + (uint64_t)p.n_combine * 4);
   l.total = off;
   return l;
 }
