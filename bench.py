@@ -53,6 +53,18 @@ def workload_figures(inp, cross=False):
     w = inp.workload
     L = inp.prefix_lengths
     total_L = int(L.sum())
+    if inp.cu_tree is not None:
+        # trees of T_b nodes: 4*d flops per (query row, prefix or tree key) pair of each
+        # sequence; bytes as below with N = sum T_b nodes
+        Tb = np.diff(inp.cu_tree).astype(np.int64)
+        N = int(Tb.sum())
+        rows = N * w.num_q_heads
+        kv_bytes = 4 * total_L * w.num_kv_heads * w.head_dim
+        flops = int(sum(4 * int(t) * w.num_q_heads * w.head_dim * (int(l) + int(t)) for t, l in zip(Tb, L)))
+        tree_bytes = 4 * N * w.num_kv_heads * w.head_dim
+        step_bytes = kv_bytes + tree_bytes + 4 * rows * w.head_dim + 4 * rows
+        return dict(total_L=total_L, step_bytes=step_bytes, step_flops=flops, partials_flops=flops,
+                    partials_bytes=kv_bytes + tree_bytes + 2 * rows * w.head_dim, kv_bytes=kv_bytes, rows=rows)
     if cross:
         # prefix-only attention: 4*d flops per (query row, prefix key); bytes: the prefix
         # K/V, the queries, out and lse
@@ -82,7 +94,9 @@ def config_of(inp, l2_note):
     return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
             "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "tree_size": w.tree_size,
             "tree": w.tree, "prefix_len": int(L[0]) if len(set(L.tolist())) == 1 else "ragged",
-            "total_prefix_len": int(L.sum()), "seed": inp.seed, "l2": l2_note}
+            "total_prefix_len": int(L.sum()), "seed": inp.seed, "l2": l2_note,
+            **({"tree_sizes": f"T_b ~ U{{{w.tree_size_range[0]}..{w.tree_size_range[1]}}}, sum {inp.num_nodes}"}
+               if w.tree_size_range else {})}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -188,17 +202,35 @@ def recorded_traffic(workload_name):
 
 
 # ----------------------------------------------------------------------------- oracle timing
+def oracle_rows(inp, rows, cores):
+    """The fp64 oracle on the given output rows (node n, head h) -> n*H_q + h."""
+    import oracle
+    if inp.cu_tree is None:
+        return oracle.verify_attn_oracle_inputs(inp, rows=rows, nthreads=cores)
+    w = inp.workload
+    off, cu, Hq = inp.cu_tree, inp.cu_seqlens, w.num_q_heads
+    for b in range(w.batch):
+        s, e = int(off[b]), int(off[b + 1])
+        sel = rows[(rows >= s * Hq) & (rows < e * Hq)]
+        if len(sel) == 0:
+            continue
+        l0, l1 = int(cu[b]), int(cu[b + 1])
+        oracle.verify_attn_oracle(inp.q[s:e], inp.k_cache[l0:l1], inp.v_cache[l0:l1], inp.k_tree[s:e],
+                                  inp.v_tree[s:e], inp.parent[s:e], np.array([0, l1 - l0], dtype=np.int32),
+                                  num_q_heads=Hq, num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                                  tree_size=e - s, scale=inp.scale, rows=sel - s * Hq, nthreads=cores)
+
+
 def time_oracle(inp, target_s=12.0, max_rows=None):
     """Time the fp64 oracle on a bounded sample of rows with every host core; returns
     (us per full call, rows sampled, seconds, cores)."""
-    import oracle
     w = inp.workload
-    total = w.batch * w.tree_size * w.num_q_heads
+    total = inp.num_nodes * w.num_q_heads
     cores = len(os.sched_getaffinity(0))
     rng = np.random.default_rng(123)
     probe = np.sort(rng.choice(total, size=min(total, max(cores, 8)), replace=False))
     t0 = time.perf_counter()
-    oracle.verify_attn_oracle_inputs(inp, rows=probe, nthreads=cores)
+    oracle_rows(inp, probe, cores)
     t_probe = max(time.perf_counter() - t0, 1e-6)
     per_row = t_probe / len(probe)
     n = int(min(total, max(len(probe), target_s / per_row)))
@@ -206,7 +238,7 @@ def time_oracle(inp, target_s=12.0, max_rows=None):
         n = min(n, max_rows)
     rows = np.sort(rng.choice(total, size=n, replace=False))
     t0 = time.perf_counter()
-    oracle.verify_attn_oracle_inputs(inp, rows=rows, nthreads=cores)
+    oracle_rows(inp, rows, cores)
     dt = time.perf_counter() - t0
     return dt / n * total * 1e6, n, dt, cores
 
@@ -218,7 +250,7 @@ def run_reference(args):
         return 0
     w = WORKLOADS[args.workload]
     inp = make_inputs(w, seed=0)
-    total = w.batch * w.tree_size * w.num_q_heads
+    total = inp.num_nodes * w.num_q_heads
     per_step_target = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     vals = []
     n_rows = cores = None
@@ -344,6 +376,30 @@ def run_ours(args):
         partials = full_call  # noqa: F811  (the paged call has no separate partials stage)
         args.no_e2e = True
 
+    if inp.cu_tree is not None or args.rope > 0:
+        # per-sequence trees and/or in-kernel RoPE: the general entry, timed as one call
+        # (tree kernel when rotating, partials, combine)
+        if args.paged:
+            raise SystemExit("--paged with per-sequence trees or --rope is not a bench mode")
+        cu_tree_d = i32(inp.cu_tree) if inp.cu_tree is not None else None
+        topt = binding.TreeOpts(cu_tree_d.data_ptr() if cu_tree_d is not None else None,
+                                inp.num_nodes if cu_tree_d is not None else 0, float(args.rope))
+        wsb_t = binding.ex_workspace_size(dims, topt)
+        ws_t = torch.empty(wsb_t, dtype=torch.uint8, device=dev)
+
+        def full_call():  # noqa: F811
+            rc = binding.call_ex_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], None, ptr["k_tree"], ptr["v_tree"],
+                                     ptr["parent"], ptr["cu"], topt, out.data_ptr(), lse.data_ptr(), dims,
+                                     ws_t.data_ptr(), wsb_t, sp)
+            if rc:
+                raise binding.LSError(rc, "ls_verify_attn_ex")
+
+        def check_status():  # noqa: F811
+            return binding.check(dims, ws_t.data_ptr(), sp)
+
+        partials = full_call  # noqa: F811
+        args.no_e2e = True
+
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
@@ -432,6 +488,7 @@ def run_ours(args):
     if rank != 0:
         return 0
 
+    whole_call = inp.cu_tree is not None or args.rope > 0
     peaks, peak_kind = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -461,13 +518,16 @@ def run_ours(args):
                            **({"kv_layout": f"paged: {args.paged} keys per page, pages in random order"}
                               if args.paged else {}),
                            **({"attention": f"prefix-only (ls_cross_attn), {args.cross} queries per sequence"}
-                              if args.cross else {})),
+                              if args.cross else {}),
+                           **({"rope_theta": args.rope, "rope": "q and k_tree rotated in-kernel at L_b + depth"}
+                              if args.rope > 0 else {})),
             "kv_hbm_gbs": fig["kv_bytes"] / step_s / 1e9,
             "roofline_step": {"roofline_us": roof_step_s * 1e6, "frac": roof_step_s / step_s,
                               "bytes": fig["step_bytes"], "flops": fig["step_flops"]},
-            "roofline": roof, "gpu_launches": 2 * K, "plan": op.plan,
-            "kernel_timing": ("paged or cross-attention call: the roofline figure times the whole call"
-                              if (args.paged or args.cross) else
+            "roofline": roof, "gpu_launches": (3 if args.rope > 0 else 2) * K, "plan": op.plan,
+            "kernel_timing": ("paged, cross-attention, per-sequence-tree or RoPE call: the roofline figure "
+                              "times the whole call"
+                              if (args.paged or args.cross or whole_call) else
                               "partials kernel timed in K further partials-only launches after the K "
                               "steps, same L2 flush and queueing"),
             "clocks": sampler.summary(), "e2e": e2e}
@@ -491,6 +551,8 @@ def main():
                     help="time ls_cross_attn (prefix-only attention) with this many queries per sequence")
     ap.add_argument("--paged", type=int, default=0,
                     help="time ls_verify_attn_paged with pages of this many keys (no e2e figure)")
+    ap.add_argument("--rope", type=float, default=0.0,
+                    help="RoPE base: q and k_tree arrive unrotated and are rotated in-kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--spin-us", type=float, default=150.0,

@@ -179,6 +179,50 @@ LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* 
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * Per-sequence trees and in-kernel tree positions, for ls_verify_attn_ex.
+ *
+ * cu_tree: trees of different sizes. Sequence b's tree nodes are rows
+ *   [cu_tree[b], cu_tree[b+1]) of q, k_tree, v_tree, tree_parent, out and lse (all packed
+ *   by cu_tree instead of b * tree_size); dims->tree_size is then the largest tree
+ *   allowed (1..128) and the work is planned for it. cu_tree is device int32 [B+1] with
+ *   cu_tree[0] = 0, cu_tree[B] = total_nodes and 0 <= cu_tree[b+1] - cu_tree[b] <=
+ *   tree_size; a sequence may have no node. tree_parent holds each tree's own local
+ *   indices (-1 for its root, node 0). A device cu_tree that breaks these rules is
+ *   reported as LS_ERR_LENGTHS by ls_verify_attn_check (its sequences get no output).
+ *   NULL: every sequence has tree_size nodes and total_nodes is ignored.
+ *
+ * rope_theta > 0: q and k_tree arrive without rotary position embedding and the
+ *   library applies it (RoFormer, listed under "Builds on" on the mlsanity page): node i
+ *   of sequence b sits at position L_b + depth(i) (the root right after the prefix,
+ *   siblings at one position), and each pair (x[e], x[e + d/2]) of a head is rotated by
+ *   the angle position * rope_theta^(-2e/d) (the half-split pairing of the Llama and Qwen
+ *   models; rope_theta is the model's base, e.g. 10000, 500000 or 1000000). The rotated
+ *   values are rounded to bf16, as a caller's own rotation would leave them, and held in
+ *   the workspace; v_tree and the cached keys (rotated when they were written) are read
+ *   as they are. rope_theta = 0: q and k_tree are already rotated.
+ */
+typedef struct {
+  const int32_t* cu_tree;
+  int32_t total_nodes;
+  double rope_theta;
+} ls_tree_opts;
+
+/*
+ * The general entry: ls_verify_attn over a packed (paged == NULL) or paged K/V cache,
+ * with per-sequence trees and in-kernel RoPE as `tree` asks (tree == NULL: neither).
+ * Arguments, results and errors are those of ls_verify_attn / ls_verify_attn_paged;
+ * with cu_tree, the tree tensors, out and lse have total_nodes rows. The workspace
+ * must hold ls_verify_attn_ex_workspace_size(dims, tree) bytes (more than
+ * ls_verify_attn_workspace_size when rope_theta > 0); ls_verify_attn_check(dims, ...)
+ * reads the call's device status.
+ */
+LS_API size_t ls_verify_attn_ex_workspace_size(const ls_verify_dims* dims, const ls_tree_opts* tree);
+LS_API int ls_verify_attn_ex(const void* q, const void* k_cache, const void* v_cache, const ls_paged_kv* paged,
+                             const void* k_tree, const void* v_tree, const int32_t* tree_parent,
+                             const int32_t* cu_seqlens, const ls_tree_opts* tree, void* out, float* lse,
+                             const ls_verify_dims* dims, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Prefix-only attention: the draft model's cross-attention over the target model's KV
  * cache (LongSpec, gist.science summary, section 2A, "Cross-Attention mit geteiltem
  * KV-Cache": the draft reads the target's cache directly, so long contexts cost it no

@@ -98,6 +98,32 @@ def verify_attn_oracle_inputs(inp, rows=None, nthreads: int = 0, scale=None):
                               rows=rows, nthreads=nthreads)
 
 
+def verify_attn_oracle_packed(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, node_offsets,
+                              *, num_q_heads: int, num_kv_heads: int, head_dim: int, scale: float,
+                              nthreads: int = 0):
+    """Trees of different sizes: sequence b's nodes are rows [off[b], off[b+1]) of q,
+    k_tree, v_tree and parent. Each sequence is its own one-sequence problem with
+    T_b = off[b+1] - off[b] nodes. Returns (out [N*H_q, d], lse [N*H_q]) in packed
+    row order (node n, head h) -> n*H_q + h."""
+    off = np.asarray(node_offsets, dtype=np.int64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    N = int(off[-1])
+    out = np.zeros((N * num_q_heads, head_dim))
+    lse = np.zeros(N * num_q_heads)
+    for b in range(len(off) - 1):
+        s, e = int(off[b]), int(off[b + 1])
+        if e == s:
+            continue
+        l0, l1 = int(cu[b]), int(cu[b + 1])
+        o, l_ = verify_attn_oracle(q[s:e], k_cache[l0:l1], v_cache[l0:l1], k_tree[s:e], v_tree[s:e],
+                                   parent[s:e], np.array([0, l1 - l0], dtype=np.int32),
+                                   num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
+                                   tree_size=e - s, scale=scale, nthreads=nthreads)
+        out[s * num_q_heads:e * num_q_heads] = o
+        lse[s * num_q_heads:e * num_q_heads] = l_
+    return out, lse
+
+
 def softmax_keyset(q_row, keys, vals, scale: float):
     """One fp64 softmax of a bf16 query row over bf16 key/value rows [n, d]."""
     lib = _load()
@@ -117,5 +143,5 @@ def check_trees(parent, B: int, T: int) -> bool:
     return _load().oracle_check_trees(_ptr(par), B, T) == 0
 
 
-__all__ = ["verify_attn_oracle", "verify_attn_oracle_inputs", "softmax_keyset", "check_trees",
+__all__ = ["verify_attn_oracle", "verify_attn_oracle_inputs", "verify_attn_oracle_packed", "softmax_keyset", "check_trees",
            "max_threads", "OracleError"]

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3:
 EXPORTED = ("ls_verify_attn", "ls_verify_attn_partials", "ls_verify_attn_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
             "ls_verify_attn_plan", "ls_verify_attn_static", "ls_verify_attn_paged", "ls_cross_attn",
-            "ls_cross_attn_workspace_size")
+            "ls_cross_attn_workspace_size", "ls_verify_attn_ex", "ls_verify_attn_ex_workspace_size")
 
 
 class LSError(RuntimeError):
@@ -40,6 +40,11 @@ class LSError(RuntimeError):
 class PagedKV(ctypes.Structure):
     _fields_ = [("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
                 ("num_pages", ctypes.c_int64), ("page_table", ctypes.c_void_p)]
+
+
+class TreeOpts(ctypes.Structure):
+    """ls_tree_opts: per-sequence trees (cu_tree, device address) and in-kernel RoPE."""
+    _fields_ = [("cu_tree", ctypes.c_void_p), ("total_nodes", ctypes.c_int32), ("rope_theta", ctypes.c_double)]
 
 
 class Dims(ctypes.Structure):
@@ -76,6 +81,12 @@ def load_library(path: str = LIB_PATH):
     lib.ls_cross_attn.restype = ctypes.c_int
     lib.ls_cross_attn_workspace_size.argtypes = [D]
     lib.ls_cross_attn_workspace_size.restype = ctypes.c_size_t
+    T = ctypes.POINTER(TreeOpts)
+    lib.ls_verify_attn_ex.argtypes = [P, P, P, ctypes.POINTER(PagedKV), P, P, P, P, T, P, P, D, P,
+                                      ctypes.c_size_t, P]
+    lib.ls_verify_attn_ex.restype = ctypes.c_int
+    lib.ls_verify_attn_ex_workspace_size.argtypes = [D, T]
+    lib.ls_verify_attn_ex_workspace_size.restype = ctypes.c_size_t
     lib.ls_verify_attn_static.argtypes = [P, P, P, P, P, P, P, P, P, D, P]
     lib.ls_verify_attn_static.restype = ctypes.c_int
     lib.ls_verify_attn_workspace_size.argtypes = [D]
@@ -142,6 +153,20 @@ def call_paged_raw(q, k_pages, v_pages, paged: PagedKV, k_tree, v_tree, parent, 
     return int(load_library().ls_verify_attn_paged(q, k_pages, v_pages, ctypes.byref(paged), k_tree, v_tree,
                                                    parent, cu_seqlens, out, lse, ctypes.byref(dims), workspace,
                                                    workspace_bytes, stream))
+
+
+def ex_workspace_size(dims: Dims, tree: Optional[TreeOpts]) -> int:
+    return int(load_library().ls_verify_attn_ex_workspace_size(ctypes.byref(dims),
+                                                               None if tree is None else ctypes.byref(tree)))
+
+
+def call_ex_raw(q, k_cache, v_cache, paged: Optional[PagedKV], k_tree, v_tree, parent, cu_seqlens,
+                tree: Optional[TreeOpts], out, lse, dims: Dims, workspace, workspace_bytes: int, stream) -> int:
+    """ls_verify_attn_ex (paged cache, per-sequence trees, in-kernel RoPE) on raw device addresses."""
+    return int(load_library().ls_verify_attn_ex(q, k_cache, v_cache, None if paged is None else ctypes.byref(paged),
+                                                k_tree, v_tree, parent, cu_seqlens,
+                                                None if tree is None else ctypes.byref(tree), out, lse,
+                                                ctypes.byref(dims), workspace, workspace_bytes, stream))
 
 
 def cross_workspace_size(dims: Dims) -> int:

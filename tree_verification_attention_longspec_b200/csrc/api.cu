@@ -59,12 +59,27 @@ int check_dims(const ls_verify_dims* d) {
   return LS_OK;
 }
 
+// Checks the per-sequence tree options; nullptr means uniform trees, no RoPE.
+int check_tree(const ls_verify_dims* d, const ls_tree_opts* t) {
+  if (t == nullptr) return LS_OK;
+  if (t->cu_tree != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(t->cu_tree) & 3u) != 0) return LS_ERR_INVALID_ARG;
+    if (t->total_nodes < 0 || (long long)t->total_nodes > (long long)d->batch * d->tree_size)
+      return LS_ERR_INVALID_ARG;
+  }
+  if (!(t->rope_theta >= 0.0) || !std::isfinite(t->rope_theta)) return LS_ERR_INVALID_ARG;
+  if (t->rope_theta > 0.0 && t->rope_theta <= 1.0) return LS_ERR_INVALID_ARG;  // a base above 1
+  return LS_OK;
+}
+
 // Chooses the chunk length C (in 128-key blocks) that minimises the estimated time of
 // the partials kernel: waves of `slots` CTAs, each wave as long as its longest chunk
 // plus a fixed per-chunk cost for loading Q and writing the partial. A sequence's key
 // list is its prefix blocks plus one tree block.
-int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true) {
+int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_tree_opts* tree = nullptr) {
   int rc = check_dims(d);
+  if (rc != LS_OK) return rc;
+  rc = check_tree(d, tree);
   if (rc != LS_OK) return rc;
   int sms = 0, major = 0;
   rc = device_info(&sms, &major);
@@ -79,6 +94,8 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true) {
   q.T = d->tree_size;
   q.g = q.Hq / q.Hkv;
   q.rows = q.T * q.g;
+  q.N = tree != nullptr && tree->cu_tree != nullptr ? tree->total_nodes : q.B * q.T;
+  q.rope = with_tree && tree != nullptr && tree->rope_theta > 0.0 ? 1 : 0;
   if (q.g > ls::kUnitRows) return LS_ERR_UNSUPPORTED;
   q.tpu = ls::kUnitRows / q.g;
   q.rg = ls::ceil_div(q.T, q.tpu);
@@ -158,13 +175,14 @@ int ls_verify_attn_plan(const ls_verify_dims* dims, int32_t* partials_ctas, int3
 
 namespace {
 
-// The partials stage for a packed (pg == nullptr) or paged K/V cache; arguments checked.
+// The partials stage for a packed (pg == nullptr) or paged K/V cache, after the tree
+// kernel when RoPE is asked for; arguments checked.
 int run_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree, const void* v_tree,
                  const int32_t* tree_parent, const int32_t* cu_seqlens, const ls_verify_dims* dims,
                  const ls_paged_kv* pg, void* workspace, size_t workspace_bytes, void* stream,
-                 bool with_tree = true) {
+                 bool with_tree = true, const ls_tree_opts* tree = nullptr) {
   Plan p;
-  int rc = make_plan(dims, &p, with_tree);
+  int rc = make_plan(dims, &p, with_tree, tree);
   if (rc != LS_OK) return rc;
   if (q == nullptr || !aligned16(q) || cu_seqlens == nullptr || !aligned4(cu_seqlens)) return LS_ERR_INVALID_ARG;
   if (with_tree) {
@@ -211,6 +229,8 @@ int run_partials(const void* q, const void* k_cache, const void* v_cache, const 
   pa.v_tree = static_cast<const uint16_t*>(with_tree ? v_tree : v_cache);
   pa.parent = tree_parent;
   pa.cu = cu_seqlens;
+  pa.cu_tree = tree != nullptr ? tree->cu_tree : nullptr;
+  pa.after_prep = 0;
   pa.page_table = pg ? pg->page_table : nullptr;
   pa.page_size = pg ? pg->page_size : 0;
   pa.max_pages = pg ? pg->max_pages_per_seq : 0;
@@ -220,7 +240,24 @@ int run_partials(const void* q, const void* k_cache, const void* v_cache, const 
   pa.p = p;
   // rows of the K/V tensors that the TMA descriptors may address (an upper bound is
   // enough: no block is ever read past the tensor)
-  if (k_cache == nullptr) kv_rows = (int64_t)p.B * p.T;
+  if (k_cache == nullptr) kv_rows = p.N;
+  if (p.rope) {
+    // rotate q and k_tree into the workspace; the partials kernel reads them from there
+    ls::TreeRopeArgs ra;
+    ra.q = pa.q;
+    ra.k_tree = pa.k_tree;
+    ra.parent = tree_parent;
+    ra.cu = cu_seqlens;
+    ra.cu_tree = pa.cu_tree;
+    ra.q_rot = reinterpret_cast<uint16_t*>(ws + lay.q_rot);
+    ra.k_rot = reinterpret_cast<uint16_t*>(ws + lay.k_rot);
+    ra.log2_theta = std::log2(tree->rope_theta);
+    ra.p = p;
+    if (ls::launch_tree_rope(ra, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LS_ERR_CUDA;
+    pa.q = ra.q_rot;
+    pa.k_tree = ra.k_rot;
+    pa.after_prep = 1;
+  }
   const cudaError_t e = ls::launch_partials(pa, kv_rows, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
@@ -242,9 +279,9 @@ int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_ca
 namespace {
 
 int run_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims, void* workspace,
-                size_t workspace_bytes, void* stream, bool with_tree) {
+                size_t workspace_bytes, void* stream, bool with_tree, const ls_tree_opts* tree = nullptr) {
   Plan p;
-  int rc = make_plan(dims, &p, with_tree);
+  int rc = make_plan(dims, &p, with_tree, tree);
   if (rc != LS_OK) return rc;
   if (out == nullptr || !aligned16(out)) return LS_ERR_INVALID_ARG;
   if (cu_seqlens == nullptr || lse == nullptr || !aligned4(cu_seqlens) || !aligned4(lse)) return LS_ERR_INVALID_ARG;
@@ -254,6 +291,7 @@ int run_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verif
   (void)cudaGetLastError();
   ls::CombineArgs ca;
   ca.cu = cu_seqlens;
+  ca.cu_tree = tree != nullptr ? tree->cu_tree : nullptr;
   ca.o_part = reinterpret_cast<const float*>(ws + lay.o_part);
   ca.lse_part = reinterpret_cast<const float*>(ws + lay.lse_part);
   ca.chunk_status = reinterpret_cast<const uint32_t*>(ws + lay.chunk_status);
@@ -320,6 +358,26 @@ int ls_verify_attn_paged(const void* q, const void* k_pages, const void* v_pages
                     workspace_bytes, stream);
   if (rc != LS_OK) return rc;
   return ls_verify_attn_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream);
+}
+
+size_t ls_verify_attn_ex_workspace_size(const ls_verify_dims* dims, const ls_tree_opts* tree) {
+  Plan p;
+  if (make_plan(dims, &p, true, tree) != LS_OK) return 0;
+  return (size_t)ls::make_layout(p).total;
+}
+
+int ls_verify_attn_ex(const void* q, const void* k_cache, const void* v_cache, const ls_paged_kv* paged,
+                      const void* k_tree, const void* v_tree, const int32_t* tree_parent, const int32_t* cu_seqlens,
+                      const ls_tree_opts* tree, void* out, float* lse, const ls_verify_dims* dims, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  Plan p;
+  int rc = make_plan(dims, &p, true, tree);
+  if (rc != LS_OK) return rc;
+  if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
+  rc = run_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, paged, workspace,
+                    workspace_bytes, stream, true, tree);
+  if (rc != LS_OK) return rc;
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, true, tree);
 }
 
 int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void* stream) {

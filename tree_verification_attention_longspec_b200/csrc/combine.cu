@@ -8,7 +8,8 @@
 //   M = max_x l_x,  w_x = 2^(l_x - M),  out = sum_x w_x o_x / sum_x w_x,
 //   lse = (M + log2 sum_x w_x) * ln 2   (natural log, scale included).
 // One warp per output row (tree node i of sequence b, query head h); lanes split the
-// head dimension. The kernel is launched as a programmatic dependent of the partials
+// head dimension. Rows are enumerated as if every sequence had T nodes; with
+// per-sequence trees (cu_tree) the rows past a sequence's own tree have no output. The kernel is launched as a programmatic dependent of the partials
 // kernel and waits for its results with griddepcontrol.wait. It uses no shared memory
 // beyond a status word, so one of its CTAs fits beside a partials CTA on an SM and is
 // ready when that grid ends.
@@ -34,11 +35,17 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   const int64_t row = (int64_t)blockIdx.x * kMergeRows + warp;
   const bool has_row = row < n_rows;
   int n = 0, cbase = 0, rl = 0;
-  bool lengths_ok = false;
+  int64_t out_row = 0;
+  bool lengths_ok = false, writes = false;
+  uint32_t err = 0u;
   if (has_row) {
     const int tok = (int)(row / p.Hq), h = (int)(row % p.Hq);
     const int b = tok / p.T, i = tok % p.T;
     const int kh = h / p.g, j = h % p.g;
+    int tree_base = 0, tree_n = 0;
+    if (!tree_range(p, a.cu_tree, b, &tree_base, &tree_n)) err |= kErrLengths;
+    writes = i < tree_n;  // the node exists in sequence b's tree
+    out_row = (int64_t)(tree_base + i) * p.Hq + h;
     int first = 0, total = 0;
     sequence_chunks(p, a.cu, b, &first, &n, &total);
     const int32_t L = a.cu[b + 1] - a.cu[b];
@@ -54,8 +61,7 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   // the partials kernel may still be running: wait for its grid to finish
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  uint32_t err = 0u;
-  if (has_row) {
+  if (writes) {
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
@@ -111,13 +117,13 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
       err |= kErrLengths;
     }
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    uint16_t* dst = a.out + row * D + lane * E;
+    uint16_t* dst = a.out + out_row * D + lane * E;
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
       const uint32_t lo = f32_to_bf16(acc[e] * inv), hi = f32_to_bf16(acc[e + 1] * inv);
       *reinterpret_cast<uint32_t*>(dst + e) = lo | (hi << 16);
     }
-    if (lane == 0) a.lse[row] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+    if (lane == 0) a.lse[out_row] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
   }
 #pragma unroll
   for (int o2 = 16; o2 > 0; o2 >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o2);

@@ -19,6 +19,7 @@ struct PartialsArgs {
   const uint16_t* v_tree;
   const int32_t* parent;
   const int32_t* cu;
+  const int32_t* cu_tree;  // per-sequence tree offsets; nullptr: T nodes each
   // paged K/V cache: page_table[b * max_pages + i] is the physical page of keys
   // [i * page_size, (i + 1) * page_size) of sequence b; nullptr = keys packed by cu
   const int32_t* page_table;
@@ -27,12 +28,28 @@ struct PartialsArgs {
   float* o_part;
   float* lse_part;
   uint32_t* chunk_status;
+  int32_t after_prep;  // q and k_tree are written by the tree kernel launched just before
+  Plan p;
+};
+
+// The tree kernel: every node's depth, and q and k_tree rotated (RoPE) to the node's
+// position prefix length + depth.
+struct TreeRopeArgs {
+  const uint16_t* q;
+  const uint16_t* k_tree;
+  const int32_t* parent;
+  const int32_t* cu;
+  const int32_t* cu_tree;
+  uint16_t* q_rot;
+  uint16_t* k_rot;
+  double log2_theta;  // log2 of the RoPE base
   Plan p;
 };
 
 // The combine kernel: the log-sum-exp merge of every chunk's partial.
 struct CombineArgs {
   const int32_t* cu;
+  const int32_t* cu_tree;
   const float* o_part;
   const float* lse_part;
   const uint32_t* chunk_status;
@@ -63,4 +80,5 @@ __device__ __forceinline__ float warp_sum(float v) {
 namespace ls {
 cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream);  // kv_rows: rows of the K/V tensors
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+cudaError_t launch_tree_rope(const TreeRopeArgs& a, cudaStream_t stream);
 }  // namespace ls

@@ -11,6 +11,8 @@
 // that holds the tree block also attends the last prefix keys, and a sequence without
 // prefix still has one chunk. The chunk grid follows from the prefix lengths and C
 // alone, and the device recomputes it from cu_seqlens without any table in memory.
+// Trees may differ in size per sequence (cu_tree): the grid is then planned for T, the
+// largest tree allowed, and units past a sequence's own tree have no rows.
 #pragma once
 #include <stdint.h>
 
@@ -33,7 +35,9 @@ constexpr uint32_t kErrLengths = 2u;
 constexpr uint32_t kErrTimeout = 4u;
 
 struct Plan {
-  int32_t B, Hq, Hkv, d, T, g;
+  int32_t B, Hq, Hkv, d, T, g;  // T: tree nodes per sequence (the largest, with cu_tree)
+  int32_t N;           // tree nodes of the batch: B * T, or cu_tree[B]
+  int32_t rope;        // 1: q and k_tree are rotated (RoPE) by the tree kernel first
   int32_t rows;        // T * g query rows per (sequence, kv head)
   int32_t tpu;         // tree nodes per unit: floor(kUnitRows / g)
   int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
@@ -56,6 +60,23 @@ LS_HD int32_t prefix_blocks(int32_t L) { return L > 0 ? ceil_div(L, kBlockN) : 0
 LS_HD int32_t chunks_per_unit(const Plan& p, int32_t L) {
   if (p.uniform_n >= 0) return p.uniform_n;
   return ceil_div(prefix_blocks(L) + p.with_tree, p.C);
+}
+
+// Tree nodes of sequence b: rows [*base, *base + *n) of q, k_tree, v_tree, tree_parent,
+// out and lse. Without cu_tree every sequence has T nodes. A cu_tree entry that does
+// not describe a packed layout (cu_tree[0] = 0, non-decreasing, cu_tree[B] = N, at most
+// T nodes a tree) gives the sequence no node and returns false.
+LS_HD bool tree_range(const Plan& p, const int32_t* cu_tree, int32_t b, int32_t* base, int32_t* n) {
+  if (cu_tree == nullptr) {
+    *base = b * p.T;
+    *n = p.T;
+    return true;
+  }
+  const int32_t s = cu_tree[b], e = cu_tree[b + 1];
+  const bool ok = s >= 0 && e >= s && e <= p.N && e - s <= p.T && (b > 0 || s == 0) && (b < p.B - 1 || e == p.N);
+  *base = ok ? s : 0;
+  *n = ok ? e - s : 0;
+  return ok;
 }
 
 // Unit and row inside the unit of query row (tree node i, head-in-group j).
@@ -128,6 +149,8 @@ struct Layout {
   uint64_t o_part;        // float [n_chunks][kUnitRows][d]   partial out, normalised
   uint64_t lse_part;      // float [n_chunks][kUnitRows]      partial lse, log2 domain
   uint64_t chunk_status;  // u32   [n_chunks]
+  uint64_t q_rot;         // bf16  [N][Hq][d]    rotated queries (rope only)
+  uint64_t k_rot;         // bf16  [N][Hkv][d]   rotated tree keys (rope only)
   uint64_t total;
 };
 
@@ -144,6 +167,11 @@ LS_HD Layout make_layout(const Plan& p) {
   off = align256(off + (uint64_t)p.n_chunks * kUnitRows * 4);
   l.chunk_status = off;
   off = align256(off + (uint64_t)p.n_chunks * 4);
+  const uint64_t nq = p.rope ? (uint64_t)p.N * p.Hq * p.d * 2 : 0, nk = p.rope ? (uint64_t)p.N * p.Hkv * p.d * 2 : 0;
+  l.q_rot = off;
+  off = align256(off + nq);
+  l.k_rot = off;
+  off = align256(off + nk);
   l.total = off;
   return l;
 }

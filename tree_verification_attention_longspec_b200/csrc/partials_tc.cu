@@ -213,8 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   const int tail_end = paged ? n_keys - (nb - 1) * kBlockN : kBlockN;
   const bool has_tree = c.has_tree;
   const int nbt = nb + (has_tree ? 1 : 0);  // blocks, the tree block (block nb) last
-  const int tok0 = c.rgi * p.tpu;                    // first tree node of the unit
-  const int rows_here = min(p.tpu, p.T - tok0) * p.g;  // rows of the unit that exist
+  int tree_base, tree_n;  // the sequence's tree nodes (none if cu_tree is bad: the combine reports it)
+  tree_range(p, a.cu_tree, c.b, &tree_base, &tree_n);
+  const int tok0 = c.rgi * p.tpu;                       // first tree node of the unit
+  const int rows_here = min(p.tpu, tree_n - tok0) * p.g;  // rows of the unit that exist
+  if (rows_here <= 0) {  // a unit past the sequence's tree: nothing to attend for
+    if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
+    return;
+  }
   if (nbt == 0) {  // empty key range: an empty partial
     for (int r = tid; r < rows_here; r += kThreads) a.lse_part[(size_t)blockIdx.x * kUnitRows + r] = -INFINITY;
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
@@ -265,22 +271,41 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     // Ring order = consumption order: K(0), V(0), K(1), V(1), ...
     if (lane == 0) {
       const int seq_len = a.cu[c.b + 1] - a.cu[c.b];
-      // Q first: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows
-      // past the batch's last node read as zeros)
-      mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
+      // Q: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows past the
+      // batch's last node read as zeros)
+      auto load_q = [&]() {
+        mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
 #pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn)
-        tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
-                    c.b * p.T + tok0);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
+                      tree_base + tok0);
+      };
+      // When the tree kernel writes q and k_tree (rotated), this grid may start before
+      // that grid ends: the prefix loads go ahead, Q and the tree block wait for it.
+      bool prior_done = !a.after_prep;
+      auto wait_prior = [&]() {
+        if (!prior_done) {
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          prior_done = true;
+        }
+      };
+      bool q_loaded = false;
+      if (prior_done) {
+        load_q();
+        q_loaded = true;
+      }
       int issued = 0, slot = 0, use = 0;
       bool ok = true;
       for (int j = 0; j < nbt && ok; ++j) {
-        // prefix block j, or the tree block: the sequence's T nodes (the rows after them
+        // prefix block j, or the tree block: the sequence's nodes (the rows after them
         // belong to the next sequence or lie past the tensor, read as zeros; masked)
         const bool tree = j == nb;
         int row = c.seq_offset + c.key_begin + j * kBlockN;
         if (j == nb - 1) row -= tail_shift;  // the box ends at the sequence end
-        if (tree) row = c.b * p.T;
+        if (tree) {
+          row = tree_base;
+          wait_prior();
+        }
         const bool pieces = paged && !tree;  // the block's rows come page by page
         for (int kv = 0; kv < 2; ++kv) {
           if (!mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs)) {
@@ -319,14 +344,20 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           }
           // K(0) alone first: at start-up every CTA asks for just Q and one tile, so those
           // arrive quickly instead of sharing the memory system with the whole ring's fill
+          if (issued == 1 && !q_loaded) {
+            wait_prior();
+            load_q();
+            q_loaded = true;
+          }
           if (issued == 1 && !mbar_wait_bounded(&bars->full[0], 0, abort, kTimeoutNs)) {
             ok = false;
             break;
           }
         }
       }
-      // make sure no copy is still writing shared memory when the CTA ends
-      drain_wait(&bars->q_full, 0);
+      // make sure no copy is still writing shared memory when the CTA ends (Q was
+      // issued unless the loop stopped before its first load)
+      if (q_loaded) drain_wait(&bars->q_full, 0);
       const int first = issued > C::kSlots ? issued - C::kSlots : 0;
       for (int seq = first; seq < issued; ++seq)
         drain_wait(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1);
@@ -348,9 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       // the tree of the sequence, for the tree mask; a parent outside [-1, T) is stored
       // as a value that fails the walk's checks
       if (has_tree) {
-        for (int x = tid; x < p.T; x += 256) {
-          const int32_t pp = a.parent[(size_t)c.b * p.T + x];
-          bars->parent[x] = (int16_t)(pp >= -1 && pp < p.T ? pp : kMaxTree);
+        for (int x = tid; x < tree_n; x += 256) {
+          const int32_t pp = a.parent[(size_t)tree_base + x];
+          bars->parent[x] = (int16_t)(pp >= -1 && pp < tree_n ? pp : kMaxTree);
         }
       }
     }
@@ -655,7 +686,7 @@ bool make_kv_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t row
 bool make_q_map(CUtensorMap* map, const void* base, int D, const Plan& p) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)p.g, (cuuint64_t)p.Hkv, (cuuint64_t)p.B * p.T};
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)p.g, (cuuint64_t)p.Hkv, (cuuint64_t)(p.N > 0 ? p.N : 1)};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)p.g * D * 2, (cuuint64_t)p.Hq * D * 2};
   cuuint32_t box[4] = {64, (cuuint32_t)p.g, 1, (cuuint32_t)p.tpu};
   cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -669,7 +700,7 @@ template <int D, int EMU>
 cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream) {
   TcParams P;
   P.a = a;
-  const int64_t tree_rows = (int64_t)a.p.B * a.p.T;
+  const int64_t tree_rows = a.p.N > 0 ? a.p.N : 1;
   // a paged cache is read in boxes of one page (at most 128 rows)
   const int box_rows = a.page_table != nullptr && a.page_size < kBlockN ? a.page_size : kBlockN;
   if (!make_q_map(&P.tmap_q, a.q, D, a.p) || !make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows, box_rows) ||
@@ -687,8 +718,22 @@ cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  partials_tc_kernel<D, EMU><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
-  return cudaGetLastError();
+  if (!a.after_prep) {
+    partials_tc_kernel<D, EMU><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
+    return cudaGetLastError();
+  }
+  // a programmatic dependent of the tree kernel (see the producer's wait_prior)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.p.n_chunks);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, partials_tc_kernel<D, EMU>, P);
 }
 
 }  // namespace

@@ -1,0 +1,121 @@
+// Tree positions and rotary embedding of the tree's queries and keys.
+//
+// A draft tree's nodes are new tokens: node i of sequence b follows the L_b cached
+// tokens at depth(i) steps below the root, so its position is L_b + depth(i) (the root,
+// depth 0, is the token right after the prefix; siblings share a position). The
+// attention uses rotary position embedding (RoFormer, listed under "Builds on" on the
+// mlsanity page; the evaluated Llama and Qwen models use it): q and k of a token at
+// position m are rotated pair by pair, pair e = (x[e], x[e + d/2]) (the half-split
+// pairing of those models' reference code, `rotate_half`) by the angle m * theta_e,
+// theta_e = base^(-2e/d). The cached keys were rotated when they were written; this
+// kernel rotates the tree's queries and keys, so that the attention kernels read them as
+// if the caller had done it. Results are rounded to bf16 like the caller's tensors.
+//
+// One CTA per (sequence, node slot); nodes past a sequence's tree do nothing. The
+// depth walk follows parent links through shared memory and stops at the root or at
+// the first link that is not a rooted tree's (the attention kernel reports that tree).
+// The angle is reduced modulo 2 pi in double precision and its sine and cosine taken in
+// float, so that large positions (10^5 and more) keep their precision.
+#include "ls_device.cuh"
+
+namespace ls {
+namespace {
+
+constexpr int kRopeThreads = 128;
+
+__global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a) {
+  const Plan& p = a.p;
+  // the attention kernel may begin its prefix loads now; it waits for this grid before
+  // it reads q_rot and k_rot
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int b = blockIdx.x / p.T, i = blockIdx.x % p.T;
+  int base = 0, n = 0;
+  tree_range(p, a.cu_tree, b, &base, &n);
+  if (i >= n) return;
+
+  __shared__ int32_t par[kMaxTree];
+  __shared__ float cos_s[64], sin_s[64];
+  __shared__ int32_t depth_s;
+  const int tid = threadIdx.x;
+  for (int x = tid; x < n; x += kRopeThreads) par[x] = a.parent[(size_t)base + x];
+  __syncthreads();
+  if (tid == 0) {
+    int x = i, depth = 0;
+    for (int step = 0; step < n && x > 0; ++step) {
+      const int pp = par[x];
+      if (pp < 0 || pp >= x) break;  // not a rooted tree: the attention kernel reports it
+      x = pp;
+      ++depth;
+    }
+    depth_s = depth;
+  }
+  __syncthreads();
+  const int32_t L = max(a.cu[b + 1] - a.cu[b], 0);
+  const double pos = (double)L + (double)depth_s;
+  const int half = p.d / 2;
+  if (tid < half) {
+    // theta_e = base^(-2e/d); the angle pos * theta_e reduced to [-pi, pi]
+    const double inv_freq = exp2(-(2.0 * tid / p.d) * a.log2_theta);
+    const double ang = pos * inv_freq;
+    constexpr double kTwoPiHi = 6.283185307179586232;     // 2 pi rounded to double
+    constexpr double kTwoPiLo = 2.4492935982947064e-16;   // 2 pi - kTwoPiHi
+    const double k = rint(ang * 0.15915494309189533577);  // ang / (2 pi), rounded
+    const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, ang));
+    float s, c;
+    sincosf((float)r, &s, &c);
+    cos_s[tid] = c;
+    sin_s[tid] = s;
+  }
+  __syncthreads();
+
+  // items: (head, group of 8 pairs); q heads first, then the kv heads of k_tree
+  const int groups = half / 8;
+  const int items = (p.Hq + p.Hkv) * groups;
+  const size_t node = (size_t)base + i;
+  for (int it = tid; it < items; it += kRopeThreads) {
+    const int hh = it / groups, e0 = (it % groups) * 8;
+    const uint16_t* src;
+    uint16_t* dst;
+    if (hh < p.Hq) {
+      src = a.q + (node * p.Hq + hh) * p.d;
+      dst = a.q_rot + (node * p.Hq + hh) * p.d;
+    } else {
+      src = a.k_tree + (node * p.Hkv + (hh - p.Hq)) * p.d;
+      dst = a.k_rot + (node * p.Hkv + (hh - p.Hq)) * p.d;
+    }
+    const uint4 lo = *reinterpret_cast<const uint4*>(src + e0);
+    const uint4 hi = *reinterpret_cast<const uint4*>(src + e0 + half);
+    const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w}, hw[4] = {hi.x, hi.y, hi.z, hi.w};
+    uint32_t ol[4], oh[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t rl = 0u, rh = 0u;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = e0 + 2 * w + k;
+        const float x1 = bf16_to_f32((uint16_t)(lw[w] >> (16 * k)));
+        const float x2 = bf16_to_f32((uint16_t)(hw[w] >> (16 * k)));
+        const float c = cos_s[e], s = sin_s[e];
+        const float y1 = fmaf(x1, c, -x2 * s);  // first of the pair
+        const float y2 = fmaf(x2, c, x1 * s);   // second of the pair
+        rl |= (uint32_t)f32_to_bf16(y1) << (16 * k);
+        rh |= (uint32_t)f32_to_bf16(y2) << (16 * k);
+      }
+      ol[w] = rl;
+      oh[w] = rh;
+    }
+    *reinterpret_cast<uint4*>(dst + e0) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+    *reinterpret_cast<uint4*>(dst + e0 + half) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_tree_rope(const TreeRopeArgs& a, cudaStream_t stream) {
+  const int64_t grid = (int64_t)a.p.B * a.p.T;
+  if (grid == 0) return cudaSuccess;
+  tree_rope_kernel<<<(unsigned)grid, kRopeThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ls

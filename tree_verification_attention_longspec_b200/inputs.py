@@ -8,14 +8,16 @@ Every tensor is returned as raw bf16 bit patterns (``uint16``) so the two sides 
 identical inputs. Floats are drawn as float32 from numpy's PCG64 and rounded to
 bf16 with round-to-nearest-even.
 
-Layouts (row-major, matching the C-ABI):
-  q        [B*T, H_q, d]      tree queries, token-major
+Layouts (row-major, matching the C-ABI; N = B*T tree nodes, or cu_tree[B] when the
+trees differ in size per sequence):
+  q        [N, H_q, d]        tree queries, token-major
   k_cache  [sum L_b, H_kv, d] prefix keys, sequences packed by cu_seqlens
   v_cache  [sum L_b, H_kv, d]
-  k_tree   [B*T, H_kv, d]     tree keys
-  v_tree   [B*T, H_kv, d]
-  parent   [B*T] int32        local parent index, -1 for the root (node 0)
+  k_tree   [N, H_kv, d]       tree keys
+  v_tree   [N, H_kv, d]
+  parent   [N] int32          local parent index, -1 for the root (node 0)
   cu_seqlens [B+1] int32      prefix offsets, cu[0] = 0
+  cu_tree  [B+1] int32        tree node offsets (per-sequence trees only), cu_tree[0] = 0
 
 The tree shapes follow the verification setting of the LongSpec paper ("Hybrid
 Tree Attention", gist.science summary, section 2C): a draft token tree whose
@@ -64,6 +66,8 @@ def star_tree(T: int) -> np.ndarray:
 def window_tree(rng: np.random.Generator, T: int, window: Optional[int]) -> np.ndarray:
     """parent[i] ~ U[max(0, i - window), i) for i >= 1 (window=None: U[0, i))."""
     p = np.empty(T, dtype=np.int32)
+    if T == 0:
+        return p
     p[0] = -1
     for i in range(1, T):
         lo = 0 if window is None else max(0, i - window)
@@ -73,6 +77,12 @@ def window_tree(rng: np.random.Generator, T: int, window: Optional[int]) -> np.n
 
 def bfs_tree(rng: np.random.Generator, T: int, max_children: int = 4,
              max_depth: int = 12) -> np.ndarray:
+    if T == 0:
+        return np.empty(0, dtype=np.int32)
+    return _bfs_tree(rng, T, max_children, max_depth)
+
+
+def _bfs_tree(rng: np.random.Generator, T: int, max_children: int, max_depth: int) -> np.ndarray:
     """Breadth-first tree: each dequeued node gets c ~ U{1..max_children} children,
     clipped to the nodes left and to depth <= max_depth (root depth 0). Nodes are
     numbered in BFS order, so parent[i] < i. If the frontier dies out before T nodes
@@ -117,6 +127,8 @@ class Workload:
     tree:   'uniform' (parent ~ U[0,i)), 'window8' (parent ~ U[max(0,i-8),i)),
             'bfs' (branching 1..4, depth <= 12), 'chain' or 'star'.
     input_scale: multiplier applied to the N(0,1) draws before bf16 rounding.
+    tree_sizes / tree_size_range: per-sequence trees, T_b given or T_b ~ U{lo..hi} i.i.d.
+            (tree_size is then the largest tree allowed); neither: T nodes each.
     """
     name: str
     batch: int
@@ -128,6 +140,12 @@ class Workload:
     tree: str
     input_scale: float = 1.0
     lengths: Optional[Sequence[int]] = field(default=None)  # explicit L_b, overrides prefix
+    tree_sizes: Optional[Sequence[int]] = field(default=None)
+    tree_size_range: Optional[tuple] = field(default=None)
+
+    @property
+    def ragged_trees(self) -> bool:
+        return self.tree_sizes is not None or self.tree_size_range is not None
 
     @property
     def group(self) -> int:
@@ -143,6 +161,19 @@ def draw_prefix_lengths(w: Workload, rng: np.random.Generator) -> np.ndarray:
         lo, hi = w.prefix
         return rng.integers(lo, hi + 1, size=w.batch).astype(np.int64)
     return np.full(w.batch, int(w.prefix), dtype=np.int64)
+
+
+def draw_tree_sizes(w: Workload, rng: np.random.Generator) -> Optional[np.ndarray]:
+    """T_b per sequence for per-sequence trees, else None (every tree has tree_size nodes)."""
+    if w.tree_sizes is not None:
+        t = np.asarray(w.tree_sizes, dtype=np.int64)
+        assert t.shape == (w.batch,) and t.min() >= 0 and t.max() <= w.tree_size
+        return t
+    if w.tree_size_range is not None:
+        lo, hi = w.tree_size_range
+        assert 0 <= lo <= hi <= w.tree_size
+        return rng.integers(lo, hi + 1, size=w.batch).astype(np.int64)
+    return None
 
 
 def draw_tree(kind: str, rng: np.random.Generator, T: int) -> np.ndarray:
@@ -170,6 +201,7 @@ class Inputs:
     parent: np.ndarray
     cu_seqlens: np.ndarray
     seed: int
+    cu_tree: Optional[np.ndarray] = None  # per-sequence trees: node offsets [B+1]
 
     @property
     def scale(self) -> float:
@@ -178,6 +210,17 @@ class Inputs:
     @property
     def prefix_lengths(self) -> np.ndarray:
         return np.diff(self.cu_seqlens).astype(np.int64)
+
+    @property
+    def num_nodes(self) -> int:
+        return int(self.q.shape[0])
+
+    def node_offsets(self) -> np.ndarray:
+        """cu_tree, or b * T for uniform trees."""
+        if self.cu_tree is not None:
+            return self.cu_tree
+        w = self.workload
+        return (np.arange(w.batch + 1) * w.tree_size).astype(np.int32)
 
 
 def _normal_bf16(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
@@ -190,24 +233,31 @@ def _normal_bf16(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
 def make_inputs(w: Workload, seed: int = 0) -> Inputs:
     """Draw the inputs of workload ``w``.
 
-    Structure (prefix lengths, then one tree per sequence) comes from
-    ``default_rng(seed + 1)``; tensors come from ``default_rng(seed)`` in the order
-    q, k_cache, v_cache, k_tree, v_tree.
+    Structure (prefix lengths, per-sequence tree sizes when the workload has them, then
+    one tree per sequence) comes from ``default_rng(seed + 1)``; tensors come from
+    ``default_rng(seed)`` in the order q, k_cache, v_cache, k_tree, v_tree.
     """
     srng = np.random.default_rng(seed + 1)
     L = draw_prefix_lengths(w, srng)
-    parents = [draw_tree(w.tree, srng, w.tree_size) for _ in range(w.batch)]
+    sizes = draw_tree_sizes(w, srng)
+    tb = sizes if sizes is not None else np.full(w.batch, w.tree_size, dtype=np.int64)
+    parents = [draw_tree(w.tree, srng, int(t)) for t in tb]
     parent = np.concatenate(parents).astype(np.int32)
     cu = np.zeros(w.batch + 1, dtype=np.int32)
     cu[1:] = np.cumsum(L)
     total_L = int(cu[-1])
+    cu_tree = None
+    if sizes is not None:
+        cu_tree = np.zeros(w.batch + 1, dtype=np.int32)
+        cu_tree[1:] = np.cumsum(sizes)
+    N = int(tb.sum())
 
     trng = np.random.default_rng(seed)
-    B, T, Hq, Hkv, d = w.batch, w.tree_size, w.num_q_heads, w.num_kv_heads, w.head_dim
+    Hq, Hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
     s = w.input_scale
-    q = _normal_bf16(trng, (B * T, Hq, d), s)
+    q = _normal_bf16(trng, (N, Hq, d), s)
     k_cache = _normal_bf16(trng, (total_L, Hkv, d), s)
     v_cache = _normal_bf16(trng, (total_L, Hkv, d), s)
-    k_tree = _normal_bf16(trng, (B * T, Hkv, d), s)
-    v_tree = _normal_bf16(trng, (B * T, Hkv, d), s)
-    return Inputs(w, q, k_cache, v_cache, k_tree, v_tree, parent, cu, seed)
+    k_tree = _normal_bf16(trng, (N, Hkv, d), s)
+    v_tree = _normal_bf16(trng, (N, Hkv, d), s)
+    return Inputs(w, q, k_cache, v_cache, k_tree, v_tree, parent, cu, seed, cu_tree)

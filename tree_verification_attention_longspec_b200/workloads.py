@@ -21,7 +21,12 @@ DEEP70B = Workload("70b_L128k_T128_h64x8_d128_bfs", batch=1, num_q_heads=64, num
 RAGGED = Workload("ragged_b8_L4k-32k_T64_h32x8_d128", batch=8, num_q_heads=32, num_kv_heads=8,
                   head_dim=128, tree_size=64, prefix=(4096, 32768), tree="window8")
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, QWEN7B, DEEP70B, RAGGED)}
+# Per-sequence trees: the ragged batch with T_b ~ U{16..128} nodes per sequence.
+RAGGED_TREES = Workload("ragged_trees_b8_L4k-32k_T16-128_h32x8_d128", batch=8, num_q_heads=32, num_kv_heads=8,
+                        head_dim=128, tree_size=128, prefix=(4096, 32768), tree="window8",
+                        tree_size_range=(16, 128))
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B, QWEN7B, DEEP70B, RAGGED, RAGGED_TREES)}
 # The headline workload: a Qwen2.5-7B-shaped layer at L = 64k, T = 64.
 HEADLINE = QWEN7B
 
