@@ -376,14 +376,15 @@ def run_ours(args):
         partials = full_call  # noqa: F811  (the paged call has no separate partials stage)
         args.no_e2e = True
 
-    if inp.cu_tree is not None or args.rope > 0:
+    if inp.cu_tree is not None or args.rope > 0 or args.window > 0:
         # per-sequence trees and/or in-kernel RoPE: the general entry, timed as one call
         # (tree kernel when rotating, partials, combine)
         if args.paged:
             raise SystemExit("--paged with per-sequence trees or --rope is not a bench mode")
         cu_tree_d = i32(inp.cu_tree) if inp.cu_tree is not None else None
-        topt = binding.TreeOpts(cu_tree_d.data_ptr() if cu_tree_d is not None else None,
-                                inp.num_nodes if cu_tree_d is not None else 0, float(args.rope))
+        topt = binding.TreeOpts(cu_tree=cu_tree_d.data_ptr() if cu_tree_d is not None else None,
+                                total_nodes=inp.num_nodes if cu_tree_d is not None else 0, window=args.window,
+                                rope_theta=float(args.rope))
         wsb_t = binding.ex_workspace_size(dims, topt)
         ws_t = torch.empty(wsb_t, dtype=torch.uint8, device=dev)
 
@@ -488,7 +489,7 @@ def run_ours(args):
     if rank != 0:
         return 0
 
-    whole_call = inp.cu_tree is not None or args.rope > 0
+    whole_call = inp.cu_tree is not None or args.rope > 0 or args.window > 0
     peaks, peak_kind = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -520,7 +521,8 @@ def run_ours(args):
                            **({"attention": f"prefix-only (ls_cross_attn), {args.cross} queries per sequence"}
                               if args.cross else {}),
                            **({"rope_theta": args.rope, "rope": "q and k_tree rotated in-kernel at L_b + depth"}
-                              if args.rope > 0 else {})),
+                              if args.rope > 0 else {}),
+                           **({"window": args.window} if args.window > 0 else {})),
             "kv_hbm_gbs": fig["kv_bytes"] / step_s / 1e9,
             "roofline_step": {"roofline_us": roof_step_s * 1e6, "frac": roof_step_s / step_s,
                               "bytes": fig["step_bytes"], "flops": fig["step_flops"]},
@@ -539,6 +541,81 @@ def run_ours(args):
     return 0
 
 
+def run_accept(args):
+    """Greedy acceptance (ls_tree_accept_greedy) over the workload's trees with bf16
+    logits of args.accept entries per node: one JSON line, HBM roofline of the logits read."""
+    import torch
+
+    from tree_verification_attention_longspec_b200 import binding
+    from tree_verification_attention_longspec_b200.inputs import make_accept_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    sizes = None
+    if w.tree_size_range:
+        sizes = np.random.default_rng(1).integers(w.tree_size_range[0], w.tree_size_range[1] + 1, size=w.batch)
+    inp = make_accept_inputs(w.batch, w.tree_size, args.accept, "bf16", tree=w.tree, match_prob=0.8, seed=0,
+                             tree_sizes=sizes)
+    N, V = inp.logits.shape
+    logits = torch.from_numpy(np.ascontiguousarray(inp.logits).view(np.int16)).to(dev)
+    tok = torch.from_numpy(inp.tokens).to(dev)
+    par = torch.from_numpy(inp.parent).to(dev)
+    cu = torch.from_numpy(inp.cu_tree).to(dev) if inp.cu_tree is not None else None
+    dims = binding.AcceptDims(inp.batch, inp.tree_size, V, binding.LS_DTYPE_BF16)
+    wsb = binding.accept_workspace_size(dims, N)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    alen = torch.empty(inp.batch, dtype=torch.int32, device=dev)
+    path = torch.empty(inp.batch, inp.tree_size, dtype=torch.int32, device=dev)
+    nxt = torch.empty(inp.batch, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def call():
+        rc = binding.call_accept_raw(logits.data_ptr(), tok.data_ptr(), par.data_ptr(),
+                                     cu.data_ptr() if cu is not None else None, N, alen.data_ptr(),
+                                     path.data_ptr(), nxt.data_ptr(), dims, ws.data_ptr(), wsb, sp)
+        if rc:
+            raise binding.LSError(rc, "ls_tree_accept_greedy")
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    got_len = alen.cpu().tolist()
+    K = args.steps
+    spin_cycles = int(args.spin_us * 2000)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    sampler = ClockSampler(0)
+    with sampler:
+        for k in range(K):
+            flush.zero_()
+            torch.cuda._sleep(spin_cycles)
+            ev[k][0].record(stream)
+            call()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+    ms = float(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    nbytes = N * V * 2 + 3 * N * 4 + inp.batch * (inp.tree_size + 2) * 4
+    ach = nbytes / (ms / 1000.0) / 1e9
+    line = {"metric": "greedy tree acceptance µs/call (argmax over the logits + tree walk)", "value": ms * 1000.0,
+            "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (N(0,1) logits with planted peaks; draft tokens copy the parent's peak w.p. 0.8)",
+            "config": {"workload": f"{w.name}_accept_V{V}", "batch": inp.batch, "nodes": N, "vocab": V,
+                       "l2": "flushed before every call, outside the timed events"},
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "traffic": None, "kernel": "ls_tree_accept_greedy (argmax + walk, whole call)",
+                         "peak_source": peak_kind},
+            "accept_len": got_len, "gpu_launches": 2 * K, "clocks": sampler.summary(), "e2e": None}
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -553,6 +630,10 @@ def main():
                     help="time ls_verify_attn_paged with pages of this many keys (no e2e figure)")
     ap.add_argument("--rope", type=float, default=0.0,
                     help="RoPE base: q and k_tree arrive unrotated and are rotated in-kernel")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding-window attention over the last WINDOW positions (draft self-attention)")
+    ap.add_argument("--accept", type=int, default=0,
+                    help="time greedy tree acceptance with bf16 logits of this vocabulary size instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--spin-us", type=float, default=150.0,
@@ -562,6 +643,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.accept:
+        return run_accept(args)
     return run_ours(args)
 
 

@@ -179,7 +179,7 @@ LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* 
                                 size_t workspace_bytes, void* stream);
 
 /*
- * Per-sequence trees and in-kernel tree positions, for ls_verify_attn_ex.
+ * Per-sequence trees, sliding windows and in-kernel tree positions, for ls_verify_attn_ex.
  *
  * cu_tree: trees of different sizes. Sequence b's tree nodes are rows
  *   [cu_tree[b], cu_tree[b+1]) of q, k_tree, v_tree, tree_parent, out and lse (all packed
@@ -190,6 +190,15 @@ LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* 
  *   indices (-1 for its root, node 0). A device cu_tree that breaks these rules is
  *   reported as LS_ERR_LENGTHS by ls_verify_attn_check (its sequences get no output).
  *   NULL: every sequence has tree_size nodes and total_nodes is ignored.
+ *
+ * window > 0: sliding-window attention (the draft model's self-attention keeps a window
+ *   of recent tokens; LongSpec, gist.science summary, section 2A, "Sliding-Window
+ *   Self-Attention", e.g. 512). A query at position P sees the keys at positions
+ *   P - window + 1 .. P, where prefix key j sits at position j and tree node i at
+ *   L_b + depth(i): node i sees the prefix keys j >= L_b + depth(i) + 1 - window and all
+ *   its ancestors (window >= tree_size is required, so no tree key falls outside it;
+ *   else LS_ERR_INVALID_ARG). The prefix may be the whole cache or just its last keys;
+ *   positions count from its first key. window = 0: the whole prefix.
  *
  * rope_theta > 0: q and k_tree arrive without rotary position embedding and the
  *   library applies it (RoFormer, listed under "Builds on" on the mlsanity page): node i
@@ -204,6 +213,7 @@ LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* 
 typedef struct {
   const int32_t* cu_tree;
   int32_t total_nodes;
+  int32_t window;
   double rope_theta;
 } ls_tree_opts;
 
@@ -236,8 +246,7 @@ LS_API int ls_verify_attn_ex(const void* q, const void* k_cache, const void* v_c
  *   workspace  at least ls_cross_attn_workspace_size(dims) bytes (it differs from
  *              ls_verify_attn_workspace_size: the key lists have no tree block)
  * Errors as for ls_verify_attn; ls_verify_attn_check reads its device status.
- * (The draft's sliding-window self-attention is ls_verify_attn itself: the window's
- * cache as the prefix and the new draft tokens as a chain tree.)
+ * (The draft's sliding-window self-attention is ls_verify_attn_ex with ls_tree_opts.window.)
  */
 LS_API size_t ls_cross_attn_workspace_size(const ls_verify_dims* dims);
 LS_API int ls_cross_attn(const void* q, const void* k_cache, const void* v_cache, const int32_t* cu_seqlens,
@@ -271,6 +280,50 @@ LS_API int ls_verify_attn_static(const void* q, const void* k_cache, const void*
                                  const void* k_tree, const void* v_tree,
                                  const int32_t* tree_parent, const int32_t* cu_seqlens,
                                  void* out, float* lse, const ls_verify_dims* dims, void* stream);
+
+/*
+ * Greedy acceptance of a verified tree (the step after verification; LongSpec,
+ * gist.science summary: section 2C verifies the tree in one pass, section 3 reports the
+ * mean acceptance length tau). For each sequence, starting at the root (node 0, the last
+ * token already accepted), the walk moves to the child whose draft token equals the
+ * argmax of the current node's logits (the smallest such child if several do) and stops
+ * when none does. This keeps exactly the tokens that greedy decoding of the target model
+ * would produce, so it is lossless; the argmax at the last node is the next token, and
+ * the step yields accept_len + 1 tokens. The argmax is the first index of the largest
+ * logit above -inf (NaN entries are skipped; a row without such a logit gives 0).
+ *
+ *   logits       [N, vocab] bf16 or fp32 (logits_dtype), row n = tree node n; N = B * T,
+ *                or total_nodes with cu_tree. 2-byte (bf16) / 4-byte (fp32) aligned;
+ *                rows that start on 16-byte boundaries are read with 16-byte loads.
+ *   tree_tokens  device int32 [N]: the draft token of every node (node 0's is not read)
+ *   tree_parent  device int32 [N]: local parents as for ls_verify_attn
+ *   cu_tree      device int32 [B+1] (per-sequence trees, as in ls_tree_opts) or NULL
+ *   accept_len   device int32 [B]: accepted draft nodes (0..T_b-1); -1 if the sequence has
+ *                no node, its cu_tree entry is not a packed layout, or its parents are not
+ *                a rooted tree with parent[i] < i
+ *   accept_path  device int32 [B, T]: local node indices of the path, root first
+ *                (accept_len + 1 entries; the rest of the row is not written)
+ *   next_token   device int32 [B]: argmax of the last node's logits (-1 when accept_len is -1)
+ *   workspace    at least ls_tree_accept_workspace_size(dims, total_nodes) bytes, 256-byte
+ *                aligned; holds per-segment maxima between the two kernels
+ * Returns LS_OK, LS_ERR_INVALID_ARG, LS_ERR_UNSUPPORTED (tree_size > 128), LS_ERR_WORKSPACE
+ * or LS_ERR_CUDA; asynchronous on `stream`. Sampling-based (non-greedy) verification is
+ * not offered.
+ */
+enum { LS_DTYPE_BF16 = 0, LS_DTYPE_F32 = 1 };
+
+typedef struct {
+  int32_t batch;         /* B >= 1 */
+  int32_t tree_size;     /* T: nodes per tree (the largest, with cu_tree), 1..128 */
+  int32_t vocab;         /* logits per node >= 1 */
+  int32_t logits_dtype;  /* LS_DTYPE_BF16 or LS_DTYPE_F32 */
+} ls_accept_dims;
+
+LS_API size_t ls_tree_accept_workspace_size(const ls_accept_dims* dims, int32_t total_nodes);
+LS_API int ls_tree_accept_greedy(const void* logits, const int32_t* tree_tokens, const int32_t* tree_parent,
+                                 const int32_t* cu_tree, int32_t total_nodes, int32_t* accept_len,
+                                 int32_t* accept_path, int32_t* next_token, const ls_accept_dims* dims,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Waits for `stream`, then reads the device-side status that the last ls_verify_attn

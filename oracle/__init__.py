@@ -124,6 +124,50 @@ def verify_attn_oracle_packed(q, k_cache, v_cache, k_tree, v_tree, parent, cu_se
     return out, lse
 
 
+def verify_attn_oracle_window(q, k_cache, v_cache, k_tree, v_tree, parent, cu_seqlens, node_offsets, *,
+                              num_q_heads: int, num_kv_heads: int, head_dim: int, scale: float, window: int,
+                              rows=None):
+    """Sliding-window attention (LongSpec, gist.science summary, section 2A): a query at
+    position P sees the keys at positions P - window + 1 .. P. Prefix key j of sequence b
+    sits at position j and tree node i at L_b + depth(i), so row (node i, head h) attends
+    the prefix keys j >= L_b + depth(i) + 1 - window and the tree nodes a on its root path
+    with depth(i) - depth(a) < window. Each row is one fp64 softmax over that explicit key
+    list (``softmax_keyset``). Rows are packed (node n, head h) -> n*H_q + h; rows=None
+    computes all of them. Returns (out [n, d], lse [n])."""
+    from .tree_positions import tree_depth_walk
+    off = np.asarray(node_offsets, dtype=np.int64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    g = num_q_heads // num_kv_heads
+    N = int(off[-1])
+    rows = np.arange(N * num_q_heads) if rows is None else np.asarray(rows, dtype=np.int64)
+    seq_of = np.searchsorted(off, np.arange(N), side="right") - 1
+    depth = np.zeros(N, dtype=np.int64)
+    for b in range(len(off) - 1):
+        if off[b + 1] > off[b]:
+            depth[off[b]:off[b + 1]] = tree_depth_walk(parent[off[b]:off[b + 1]])
+    out = np.zeros((len(rows), head_dim))
+    lse = np.zeros(len(rows))
+    for r_i, r in enumerate(rows):
+        n, h = divmod(int(r), num_q_heads)
+        b = int(seq_of[n])
+        i = n - int(off[b])
+        kh = h // g
+        L = int(cu[b + 1] - cu[b])
+        j0 = max(0, L + int(depth[n]) + 1 - window)
+        path = []
+        x = i
+        while True:
+            if int(depth[n]) - int(depth[int(off[b]) + x]) < window:
+                path.append(int(off[b]) + x)
+            if x == 0:
+                break
+            x = int(parent[int(off[b]) + x])
+        keys = np.concatenate([k_cache[int(cu[b]) + j0:int(cu[b + 1]), kh], k_tree[path, kh]])
+        vals = np.concatenate([v_cache[int(cu[b]) + j0:int(cu[b + 1]), kh], v_tree[path, kh]])
+        out[r_i], lse[r_i] = softmax_keyset(q[n, h], keys, vals, scale)
+    return out, lse
+
+
 def softmax_keyset(q_row, keys, vals, scale: float):
     """One fp64 softmax of a bf16 query row over bf16 key/value rows [n, d]."""
     lib = _load()
@@ -143,5 +187,6 @@ def check_trees(parent, B: int, T: int) -> bool:
     return _load().oracle_check_trees(_ptr(par), B, T) == 0
 
 
-__all__ = ["verify_attn_oracle", "verify_attn_oracle_inputs", "verify_attn_oracle_packed", "softmax_keyset", "check_trees",
+__all__ = ["verify_attn_oracle", "verify_attn_oracle_inputs", "verify_attn_oracle_packed",
+           "verify_attn_oracle_window", "softmax_keyset", "check_trees",
            "max_threads", "OracleError"]

@@ -73,6 +73,21 @@ def test_random_plans(plan_check):
         assert r.returncode == 0, r.stdout
 
 
+@pytest.mark.parametrize("window", [1, 64, 129, 512, 4096])
+def test_sliding_window_plans(plan_check, window):
+    # the attended range of every sequence and the per-row cut of every depth
+    rng = np.random.default_rng(window)
+    for _ in range(12):
+        B = int(rng.integers(1, 5))
+        T = int(rng.integers(1, min(window, 128) + 1))
+        lengths = rng.integers(0, 5000, size=B)
+        C = int(rng.integers(1, 12))
+        env = dict(os.environ, PLAN_CHECK_WINDOW=str(window))
+        r = subprocess.run([plan_check, str(B), "8", "2", str(T), str(C), "-1", *map(str, lengths)],
+                           capture_output=True, text=True, env=env)
+        assert r.returncode == 0, r.stdout
+
+
 def _declared_symbols():
     text = open(HEADER).read()
     return re.findall(r"LS_API\s+[\w\s\*]+?\b(ls_\w+)\s*\(", text)

@@ -18,15 +18,16 @@ from tree_verification_attention_longspec_b200.inputs import Workload, make_inpu
 pytestmark = pytest.mark.gpu
 
 
-def _tree_opts(inp, theta, cu_tree_dev):
-    if inp.cu_tree is None and theta == 0.0:
+def _tree_opts(inp, theta, cu_tree_dev, window=0):
+    if inp.cu_tree is None and theta == 0.0 and window == 0:
         return None
     ragged = inp.cu_tree is not None
-    return binding.TreeOpts(cu_tree_dev.data_ptr() if ragged else None, inp.num_nodes if ragged else 0,
-                            float(theta))
+    return binding.TreeOpts(cu_tree=cu_tree_dev.data_ptr() if ragged else None,
+                            total_nodes=inp.num_nodes if ragged else 0, window=window, rope_theta=float(theta))
 
 
-def _run_ex(inp, theta=0.0, page_size=None, host_lengths=True, cu_tree_dev=None, expect_rc=binding.LS_OK):
+def _run_ex(inp, theta=0.0, page_size=None, host_lengths=True, cu_tree_dev=None, expect_rc=binding.LS_OK,
+            window=0):
     """Returns (out fp64 [N*H_q, d], lse fp64 [N*H_q], device status, q after the call)."""
     w = inp.workload
     dev = to_device(inp)
@@ -36,7 +37,7 @@ def _run_ex(inp, theta=0.0, page_size=None, host_lengths=True, cu_tree_dev=None,
                                    cu_seqlens_host=inp.cu_seqlens if host_lengths else None)
     if cu_tree_dev is None and inp.cu_tree is not None:
         cu_tree_dev = torch.from_numpy(inp.cu_tree.astype(np.int32)).cuda()
-    tree = _tree_opts(inp, theta, cu_tree_dev)
+    tree = _tree_opts(inp, theta, cu_tree_dev, window)
     wsb = binding.ex_workspace_size(dims, tree)
     assert wsb > 0
     ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
@@ -67,12 +68,17 @@ def _run_ex(inp, theta=0.0, page_size=None, host_lengths=True, cu_tree_dev=None,
     return o, l_, status, q_after
 
 
-def _oracle(inp, theta=0.0):
+def _oracle(inp, theta=0.0, window=0):
     w = inp.workload
     q, kt = inp.q, inp.k_tree
     if theta > 0:
         pos = tp.tree_positions(inp.parent, inp.cu_seqlens, inp.node_offsets())
         q, kt = tp.rope_bf16(q, pos, theta), tp.rope_bf16(kt, pos, theta)
+    if window > 0:
+        return oracle.verify_attn_oracle_window(q, inp.k_cache, inp.v_cache, kt, inp.v_tree, inp.parent,
+                                                inp.cu_seqlens, inp.node_offsets(), num_q_heads=w.num_q_heads,
+                                                num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, scale=inp.scale,
+                                                window=window)
     return oracle.verify_attn_oracle_packed(q, inp.k_cache, inp.v_cache, kt, inp.v_tree, inp.parent,
                                             inp.cu_seqlens, inp.node_offsets(), num_q_heads=w.num_q_heads,
                                             num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, scale=inp.scale)
@@ -163,10 +169,47 @@ def test_bad_device_cu_tree_reported():
 def test_host_checks_of_tree_options():
     dims, keep = binding.make_dims(2, 8, 2, 64, 16, max_prefix_len=100)
     cu = torch.tensor([0, 5, 9], dtype=torch.int32, device="cuda")
-    too_many = binding.TreeOpts(cu.data_ptr(), 33, 0.0)  # more than B * T nodes
+    too_many = binding.TreeOpts(cu_tree=cu.data_ptr(), total_nodes=33)  # more than B * T nodes
     assert binding.ex_workspace_size(dims, too_many) == 0
-    assert binding.ex_workspace_size(dims, binding.TreeOpts(None, 0, 0.5)) == 0  # base <= 1
-    assert binding.ex_workspace_size(dims, binding.TreeOpts(None, 0, float("nan"))) == 0
+    assert binding.ex_workspace_size(dims, binding.TreeOpts(rope_theta=0.5)) == 0  # base <= 1
+    assert binding.ex_workspace_size(dims, binding.TreeOpts(rope_theta=float("nan"))) == 0
     plain = binding.ex_workspace_size(dims, None)
     assert plain == binding.workspace_size(dims)
-    assert binding.ex_workspace_size(dims, binding.TreeOpts(None, 0, 10000.0)) > plain
+    assert binding.ex_workspace_size(dims, binding.TreeOpts(rope_theta=10000.0)) > plain
+    assert binding.ex_workspace_size(dims, binding.TreeOpts(window=15)) == 0  # shorter than the tree
+    assert binding.ex_workspace_size(dims, binding.TreeOpts(window=-1)) == 0
+    assert 0 < binding.ex_workspace_size(dims, binding.TreeOpts(window=16)) <= plain
+
+
+# ----------------------------------------------------------------------------- sliding window
+@pytest.mark.parametrize("window,lengths", [
+    (512, [3000, 700, 0, 511]),   # full windows, one just short, no prefix, L = W - 1
+    (129, [1000, 5, 260, 129]),   # per-row cuts up to 231 keys: across two key blocks
+    (64, [64, 63, 65, 192]),      # the smallest window for 64 nodes
+])
+def test_sliding_window(window, lengths):
+    w = Workload("win", 4, 8, 2, 128, 64, 0, "window8", lengths=lengths)
+    inp = make_inputs(w, seed=31)
+    o, l_, st, _ = _run_ex(inp, window=window)
+    assert st == binding.LS_OK
+    ro, rl = _oracle(inp, window=window)
+    _assert_close(o, l_, ro, rl)
+
+
+@pytest.mark.parametrize("page_size", [16, 256])
+def test_sliding_window_paged_ragged_rope(page_size):
+    w = Workload("win_paged", 3, 28, 4, 128, 128, 0, "bfs", lengths=[4100, 300, 777], tree_sizes=[128, 37, 1])
+    inp = make_inputs(w, seed=32)
+    o, l_, st, _ = _run_ex(inp, 500000.0, page_size=page_size, window=300)
+    assert st == binding.LS_OK
+    ro, rl = _oracle(inp, 500000.0, window=300)
+    _assert_close(o, l_, ro, rl)
+
+
+def test_sliding_window_d64_device_lengths():
+    w = Workload("win64", 2, 4, 1, 64, 16, 0, "uniform", lengths=[2000, 200])
+    inp = make_inputs(w, seed=33)
+    o, l_, st, _ = _run_ex(inp, window=100, host_lengths=False)
+    assert st == binding.LS_OK
+    ro, rl = _oracle(inp, window=100)
+    _assert_close(o, l_, ro, rl)

@@ -22,7 +22,9 @@ STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3:
 EXPORTED = ("ls_verify_attn", "ls_verify_attn_partials", "ls_verify_attn_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
             "ls_verify_attn_plan", "ls_verify_attn_static", "ls_verify_attn_paged", "ls_cross_attn",
-            "ls_cross_attn_workspace_size", "ls_verify_attn_ex", "ls_verify_attn_ex_workspace_size")
+            "ls_cross_attn_workspace_size", "ls_verify_attn_ex", "ls_verify_attn_ex_workspace_size",
+            "ls_tree_accept_greedy", "ls_tree_accept_workspace_size")
+LS_DTYPE_BF16, LS_DTYPE_F32 = 0, 1
 
 
 class LSError(RuntimeError):
@@ -43,8 +45,15 @@ class PagedKV(ctypes.Structure):
 
 
 class TreeOpts(ctypes.Structure):
-    """ls_tree_opts: per-sequence trees (cu_tree, device address) and in-kernel RoPE."""
-    _fields_ = [("cu_tree", ctypes.c_void_p), ("total_nodes", ctypes.c_int32), ("rope_theta", ctypes.c_double)]
+    """ls_tree_opts: per-sequence trees (cu_tree, device address), sliding window, in-kernel RoPE."""
+    _fields_ = [("cu_tree", ctypes.c_void_p), ("total_nodes", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double)]
+
+
+class AcceptDims(ctypes.Structure):
+    """ls_accept_dims of the greedy acceptance call."""
+    _fields_ = [("batch", ctypes.c_int32), ("tree_size", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("logits_dtype", ctypes.c_int32)]
 
 
 class Dims(ctypes.Structure):
@@ -87,6 +96,11 @@ def load_library(path: str = LIB_PATH):
     lib.ls_verify_attn_ex.restype = ctypes.c_int
     lib.ls_verify_attn_ex_workspace_size.argtypes = [D, T]
     lib.ls_verify_attn_ex_workspace_size.restype = ctypes.c_size_t
+    A = ctypes.POINTER(AcceptDims)
+    lib.ls_tree_accept_workspace_size.argtypes = [A, ctypes.c_int32]
+    lib.ls_tree_accept_workspace_size.restype = ctypes.c_size_t
+    lib.ls_tree_accept_greedy.argtypes = [P, P, P, P, ctypes.c_int32, P, P, P, A, P, ctypes.c_size_t, P]
+    lib.ls_tree_accept_greedy.restype = ctypes.c_int
     lib.ls_verify_attn_static.argtypes = [P, P, P, P, P, P, P, P, P, D, P]
     lib.ls_verify_attn_static.restype = ctypes.c_int
     lib.ls_verify_attn_workspace_size.argtypes = [D]
@@ -167,6 +181,18 @@ def call_ex_raw(q, k_cache, v_cache, paged: Optional[PagedKV], k_tree, v_tree, p
                                                 k_tree, v_tree, parent, cu_seqlens,
                                                 None if tree is None else ctypes.byref(tree), out, lse,
                                                 ctypes.byref(dims), workspace, workspace_bytes, stream))
+
+
+def accept_workspace_size(dims: AcceptDims, total_nodes: int) -> int:
+    return int(load_library().ls_tree_accept_workspace_size(ctypes.byref(dims), int(total_nodes)))
+
+
+def call_accept_raw(logits, tokens, parent, cu_tree, total_nodes: int, accept_len, accept_path, next_token,
+                    dims: AcceptDims, workspace, workspace_bytes: int, stream) -> int:
+    """ls_tree_accept_greedy on raw device addresses; returns the status code."""
+    return int(load_library().ls_tree_accept_greedy(logits, tokens, parent, cu_tree, int(total_nodes), accept_len,
+                                                    accept_path, next_token, ctypes.byref(dims), workspace,
+                                                    workspace_bytes, stream))
 
 
 def cross_workspace_size(dims: Dims) -> int:

@@ -67,6 +67,8 @@ int check_tree(const ls_verify_dims* d, const ls_tree_opts* t) {
     if (t->total_nodes < 0 || (long long)t->total_nodes > (long long)d->batch * d->tree_size)
       return LS_ERR_INVALID_ARG;
   }
+  // a window shorter than the tree would also cut tree keys: not offered
+  if (t->window < 0 || (t->window > 0 && t->window < d->tree_size)) return LS_ERR_INVALID_ARG;
   if (!(t->rope_theta >= 0.0) || !std::isfinite(t->rope_theta)) return LS_ERR_INVALID_ARG;
   if (t->rope_theta > 0.0 && t->rope_theta <= 1.0) return LS_ERR_INVALID_ARG;  // a base above 1
   return LS_OK;
@@ -96,6 +98,7 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_
   q.rows = q.T * q.g;
   q.N = tree != nullptr && tree->cu_tree != nullptr ? tree->total_nodes : q.B * q.T;
   q.rope = with_tree && tree != nullptr && tree->rope_theta > 0.0 ? 1 : 0;
+  q.window = with_tree && tree != nullptr ? tree->window : 0;
   if (q.g > ls::kUnitRows) return LS_ERR_UNSUPPORTED;
   q.tpu = ls::kUnitRows / q.g;
   q.rg = ls::ceil_div(q.T, q.tpu);
@@ -108,7 +111,7 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_
   for (int b = 0; b < q.B; ++b) {
     const int32_t L = d->cu_seqlens_host ? d->cu_seqlens_host[b + 1] - d->cu_seqlens_host[b]
                                          : d->max_prefix_len;
-    blocks[b] = ls::prefix_blocks(L) + (with_tree ? 1 : 0);  // prefix blocks and the tree block
+    blocks[b] = ls::prefix_blocks(ls::attended_len(q, L)) + (with_tree ? 1 : 0);  // prefix blocks, tree block
     if (blocks[b] > max_blocks) max_blocks = blocks[b];
   }
   const long long units = (long long)q.Hkv * q.rg;
@@ -298,6 +301,8 @@ int run_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verif
   ca.out = static_cast<uint16_t*>(out);
   ca.lse = lse;
   ca.status = reinterpret_cast<uint32_t*>(ws + lay.status);
+  // the partials kernel ran just before unless a prefix-only call had no key at all
+  ca.after_partials = with_tree || p.n_chunks > 0 ? 1 : 0;
   ca.p = p;
   if (ls::launch_combine(ca, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;

@@ -52,7 +52,7 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
     // the device lengths must give the chunk grid the host planned (else some keys were
     // never attended): same chunk count, and a uniform plan long enough for this L
     lengths_ok = L >= 0 && total == p.n_chunks &&
-                 (p.uniform_n < 0 || (int64_t)prefix_blocks(L) + p.with_tree <= (int64_t)p.uniform_n * p.C);
+                 (p.uniform_n < 0 || (int64_t)prefix_blocks(attended_len(p, L)) + p.with_tree <= (int64_t)p.uniform_n * p.C);
     int32_t u, r;
     unit_row(p, i, j, &u, &r);
     rl = r;
@@ -145,7 +145,7 @@ cudaError_t launch_d(const CombineArgs& a, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.after_partials ? 1 : 0;  // else an ordinary launch (it reads cu before its wait)
   return cudaLaunchKernelEx(&cfg, combine_kernel<D>, a);
 }
 

@@ -56,6 +56,7 @@ struct CombineArgs {
   uint16_t* out;
   float* lse;
   uint32_t* status;
+  int32_t after_partials;  // launched right after the partials kernel: a programmatic dependent
   Plan p;
 };
 

@@ -38,6 +38,7 @@ struct Plan {
   int32_t B, Hq, Hkv, d, T, g;  // T: tree nodes per sequence (the largest, with cu_tree)
   int32_t N;           // tree nodes of the batch: B * T, or cu_tree[B]
   int32_t rope;        // 1: q and k_tree are rotated (RoPE) by the tree kernel first
+  int32_t window;      // > 0: sliding window of this many positions; 0: the whole prefix
   int32_t rows;        // T * g query rows per (sequence, kv head)
   int32_t tpu;         // tree nodes per unit: floor(kUnitRows / g)
   int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
@@ -55,11 +56,38 @@ LS_HD int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
 // 128-key blocks of a prefix of L keys
 LS_HD int32_t prefix_blocks(int32_t L) { return L > 0 ? ceil_div(L, kBlockN) : 0; }
 
-// chunks of one (sequence, kv head, unit) for a prefix of L keys: its prefix blocks
-// and (with_tree) the tree block, C per chunk
+// Sliding window (draft self-attention; LongSpec, gist.science summary, section 2A): a
+// query at position P sees the keys at positions P - window + 1 .. P. Node i sits at
+// position L + depth(i) and prefix key j at position j, so the root sees the prefix keys
+// from L + 1 - window on and deeper nodes fewer (a per-row cut, `window_cut`). The
+// attended range [window_start, L) is what every row of the sequence may need, started
+// on a 128-key boundary (so that a block never straddles two pages of a paged cache);
+// the keys before the exact start are cut for every row. window = 0: the whole prefix.
+LS_HD int32_t window_start(const Plan& p, int32_t L) {
+  if (p.window <= 0 || L <= 0) return 0;
+  const int32_t s = L + 1 - p.window;
+  return s <= 0 ? 0 : s / kBlockN * kBlockN;
+}
+
+// prefix keys of a sequence of L keys that its rows may attend
+LS_HD int32_t attended_len(const Plan& p, int32_t L) {
+  if (L <= 0) return 0;
+  return L - window_start(p, L);
+}
+
+// The first attended key (index into [window_start, L)) that a row at tree depth `depth`
+// may see; 0 without a window.
+LS_HD int32_t window_cut(const Plan& p, int32_t L, int32_t depth) {
+  if (p.window <= 0 || L <= 0) return 0;
+  const int32_t c = L + depth + 1 - p.window - window_start(p, L);
+  return c > 0 ? c : 0;
+}
+
+// chunks of one (sequence, kv head, unit) for a prefix of L keys: its attended prefix
+// blocks and (with_tree) the tree block, C per chunk
 LS_HD int32_t chunks_per_unit(const Plan& p, int32_t L) {
   if (p.uniform_n >= 0) return p.uniform_n;
-  return ceil_div(prefix_blocks(L) + p.with_tree, p.C);
+  return ceil_div(prefix_blocks(attended_len(p, L)) + p.with_tree, p.C);
 }
 
 // Tree nodes of sequence b: rows [*base, *base + *n) of q, k_tree, v_tree, tree_parent,
@@ -87,8 +115,9 @@ LS_HD void unit_row(const Plan& p, int32_t i, int32_t j, int32_t* unit, int32_t*
 
 struct ChunkCoord {
   int32_t b, kh, rgi, split, n_split;  // sequence, kv head, unit, split index, splits of unit
-  int32_t key_begin, key_end;          // prefix key range of the chunk
-  int32_t seq_offset;                  // cu_seqlens[b]
+  int32_t key_begin, key_end;          // attended key range of the chunk (from window_start)
+  int32_t key_skip;                    // window_start: prefix keys before the attended range
+  int32_t seq_offset;                  // cu_seqlens[b] + key_skip
   bool has_tree;                       // the chunk also attends the tree block
   bool valid;
 };
@@ -111,8 +140,9 @@ LS_HD ChunkCoord locate_chunk(const Plan& p, const int32_t* cu, int32_t cid) {
       c.rgi = u % p.rg;
       c.split = local % n;
       c.n_split = n;
-      c.seq_offset = cu[b];
-      const int32_t Lc = L < 0 ? 0 : L;
+      c.key_skip = window_start(p, L);
+      c.seq_offset = cu[b] + c.key_skip;
+      const int32_t Lc = attended_len(p, L);
       const int32_t v0 = c.split * p.C, v1 = v0 + p.C;  // blocks [v0, v1) of the key list
       const int32_t kb = v0 * kBlockN, ke = v1 * kBlockN;
       c.key_begin = kb < Lc ? kb : Lc;

@@ -213,6 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   const int tail_end = paged ? n_keys - (nb - 1) * kBlockN : kBlockN;
   const bool has_tree = c.has_tree;
   const int nbt = nb + (has_tree ? 1 : 0);  // blocks, the tree block (block nb) last
+  const int seq_len = a.cu[c.b + 1] - a.cu[c.b];
+  // sliding window: a row at depth d sees the attended keys from window_cut(d) on, which
+  // is below 2 * 128, so only the chunks that start there cut rows individually
+  const bool win_rows = p.window > 0 && nb > 0 && c.key_begin < 2 * kBlockN;
   int tree_base, tree_n;  // the sequence's tree nodes (none if cu_tree is bad: the combine reports it)
   tree_range(p, a.cu_tree, c.b, &tree_base, &tree_n);
   const int tok0 = c.rgi * p.tpu;                       // first tree node of the unit
@@ -270,7 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     // ------------------------------------------------------------------ TMA producer
     // Ring order = consumption order: K(0), V(0), K(1), V(1), ...
     if (lane == 0) {
-      const int seq_len = a.cu[c.b + 1] - a.cu[c.b];
       // Q: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows past the
       // batch's last node read as zeros)
       auto load_q = [&]() {
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             const int bh = a.page_size < kBlockN ? a.page_size : kBlockN;
             const int n_pages = (seq_len + a.page_size - 1) / a.page_size;
             for (int pc = 0; pc < kBlockN / bh; ++pc) {
-              const int key = c.key_begin + j * kBlockN + pc * bh;
+              const int key = c.key_skip + c.key_begin + j * kBlockN + pc * bh;
               int lp = key / a.page_size;
               if (lp >= n_pages) lp = n_pages - 1;
               if (lp >= a.max_pages) lp = a.max_pages - 1;
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       fence_proxy_async_smem();
       // the tree of the sequence, for the tree mask; a parent outside [-1, T) is stored
       // as a value that fails the walk's checks
-      if (has_tree) {
+      if (has_tree || win_rows) {
         for (int x = tid; x < tree_n; x += 256) {
           const int32_t pp = a.parent[(size_t)tree_base + x];
           bars->parent[x] = (int16_t)(pp >= -1 && pp < tree_n ? pp : kMaxTree);
@@ -490,12 +493,27 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const int ur = t * 128 + row;       // row of the unit
       const bool has_row = ur < rows_here;
       const int node = tok0 + ur / p.g;   // its tree node
+      int cut = 0;                        // window: first attended key this row sees
+      if (win_rows && has_row) {
+        int x = node, depth = 0;
+        for (int step = 0; step < kMaxTree && x > 0; ++step) {
+          const int pp = bars->parent[x];
+          if (pp < 0 || pp >= x) break;  // not a rooted tree: the tree block's chunk reports it
+          x = pp;
+          ++depth;
+        }
+        cut = window_cut(p, seq_len, depth);
+      }
       bool ok = true;
       for (int j = 0; j < nbt; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], j & 1, abort, kTimeoutNs));
         if (!ok) break;
         tc_fence_after_sync();
-        const int shift = j == nb - 1 ? tail_shift : 0;    // masked leading columns
+        int shift = j == nb - 1 ? tail_shift : 0;          // masked leading columns (this row)
+        if (win_rows && j < nb) {
+          const int kb = c.key_begin + j * kBlockN - shift;  // attended key of column 0
+          shift = max(shift, min(cut - kb, kBlockN));
+        }
         const int lim = j == nb - 1 ? tail_end : kBlockN;  // columns from here on are masked
         const bool tree_blk = j == nb;                      // keys = the sequence's tree nodes
         if (tree_blk && mask_tree_scores(bars->parent, tS, has_row ? node : -1)) bars->tree_err = 1u;
@@ -535,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         const bool raise = mx > m + kRescaleThreshold;
         const bool any_raise = __any_sync(0xffffffffu, raise);
         // masked columns (-inf) and the rare blocks that raise m take the MUFU-only path
-        const bool mufu_only = EMU == 0 || shift > 0 || lim < kBlockN || tree_blk || any_raise;
+        const bool mufu_only = EMU == 0 || __any_sync(0xffffffffu, shift > 0) || lim < kBlockN || tree_blk || any_raise;
         const float m_new = raise ? mx : m;
         // a row that has seen no visible key yet (a padding row of a tree-only chunk)
         // keeps m = -inf; its P is 0 against any finite reference

@@ -261,3 +261,51 @@ def make_inputs(w: Workload, seed: int = 0) -> Inputs:
     k_tree = _normal_bf16(trng, (N, Hkv, d), s)
     v_tree = _normal_bf16(trng, (N, Hkv, d), s)
     return Inputs(w, q, k_cache, v_cache, k_tree, v_tree, parent, cu, seed, cu_tree)
+
+
+# ----------------------------------------------------------------------------- acceptance
+@dataclass
+class AcceptInputs:
+    """One greedy-acceptance step: logits of every tree node, draft tokens, tree."""
+    logits: np.ndarray            # [N, V] bf16 bits (uint16) or float32
+    tokens: np.ndarray            # [N] int32 draft tokens (node 0's unused)
+    parent: np.ndarray            # [N] int32 local parents
+    cu_tree: Optional[np.ndarray]  # [B+1] int32, or None (T nodes each)
+    batch: int
+    tree_size: int
+    vocab: int
+    dtype: str                    # "bf16" or "f32"
+
+
+def make_accept_inputs(batch: int, tree_size: int, vocab: int, dtype: str = "bf16", tree: str = "window8",
+                       match_prob: float = 0.7, seed: int = 0,
+                       tree_sizes: Optional[Sequence[int]] = None) -> AcceptInputs:
+    """Logits N(0,1) with one planted peak per node (value 8 at a random token), and draft
+    tokens that copy the parent's planted token with probability match_prob (else a
+    random token), so that walks of several steps occur. Nothing here computes an
+    argmax: the planted peak is only where the generator put the large value.
+    Structure from ``default_rng(seed + 1)``, values from ``default_rng(seed)``."""
+    srng = np.random.default_rng(seed + 1)
+    sizes = (np.full(batch, tree_size, dtype=np.int64) if tree_sizes is None
+             else np.asarray(tree_sizes, dtype=np.int64))
+    parents = [draw_tree(tree, srng, int(t)) for t in sizes]
+    parent = np.concatenate(parents).astype(np.int32) if len(parents) else np.zeros(0, np.int32)
+    N = int(sizes.sum())
+    cu_tree = None
+    if tree_sizes is not None:
+        cu_tree = np.zeros(batch + 1, dtype=np.int32)
+        cu_tree[1:] = np.cumsum(sizes)
+    vrng = np.random.default_rng(seed)
+    x = vrng.standard_normal(size=(N, vocab), dtype=np.float32)
+    peak = vrng.integers(0, vocab, size=N)
+    x[np.arange(N), peak] = 8.0
+    tokens = vrng.integers(0, vocab, size=N).astype(np.int32)
+    copy = vrng.random(N) < match_prob
+    off = 0
+    for t in sizes:
+        for i in range(1, int(t)):
+            if copy[off + i]:
+                tokens[off + i] = peak[off + parent[off + i]]
+        off += int(t)
+    logits = bf16_bits_from_f32(x) if dtype == "bf16" else x
+    return AcceptInputs(logits, tokens, parent, cu_tree, batch, tree_size, vocab, dtype)
