@@ -40,9 +40,9 @@ struct AcceptArgs {
 namespace {
 
 constexpr int kArgmaxThreads = 256;
-constexpr int kUnroll = 4;  // 16-byte loads in flight per thread
+constexpr int kUnroll = 8;  // 16-byte loads in flight per thread
 constexpr int kWalkThreads = kMaxTree;
-constexpr int kMergeBatch = 8;  // segment results loaded together by the walk kernel
+constexpr int kMergeBatch = 16;  // segment results loaded together by the walk kernel
 
 // (v, i) beats (w, j): larger value, or equal value and smaller index; NaN never wins
 __device__ __forceinline__ bool beats(float v, int i, float w, int j) { return v > w || (v == w && i < j); }

@@ -125,7 +125,12 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // P = 2^(s*cs - m) for 64 scores, packed to bf16 pairs; adds the values to (sum0, sum1).
-// EMU of every 4 pairs use the FMA-pipe exponential.
+// EMU of every 4 pairs use the FMA-pipe exponential. Every block takes this one path,
+// masked or not (one copy of the loop keeps the softmax's code small; a second, MUFU-only
+// copy for masked blocks cost 6% in time): a masked score (-inf) gives 0 on the MUFU
+// and 2^-125 on the FMA pipe, which clamps its input there, and 2^-125 is nothing next
+// to the row's own maximum term, 1 (or, in a row with no visible key yet, m stays -inf
+// and a later raise multiplies the sums by 2^-inf = 0).
 template <int EMU>
 __device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float m, uint32_t (&pk)[kHalf / 2],
                                        float& sum0, float& sum1) {
@@ -552,8 +557,6 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         }
         const bool raise = mx > m + kRescaleThreshold;
         const bool any_raise = __any_sync(0xffffffffu, raise);
-        // masked columns (-inf) and the rare blocks that raise m take the MUFU-only path
-        const bool mufu_only = EMU == 0 || __any_sync(0xffffffffu, shift > 0) || lim < kBlockN || tree_blk || any_raise;
         const float m_new = raise ? mx : m;
         // a row that has seen no visible key yet (a padding row of a tree-only chunk)
         // keeps m = -inf; its P is 0 against any finite reference
@@ -561,8 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         float sum0 = 0.f, sum1 = 0.f;
         {
           uint32_t pk[kHalf / 2];
-          if (mufu_only) make_p<0>(lo, cs, m_ref, pk, sum0, sum1);
-          else make_p<EMU>(lo, cs, m_ref, pk, sum0, sum1);
+          make_p<EMU>(lo, cs, m_ref, pk, sum0, sum1);
           if (any_raise) {
             // the maximum moved up: rescale what O_t and l hold. O_t is idle: every PV of
             // this tile issued before S_t(j) has completed (s_full), and PV_t(j) waits for
@@ -603,8 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         }
         {
           uint32_t pk[kHalf / 2];
-          if (mufu_only) make_p<0>(hi, cs, m_ref, pk, sum0, sum1);
-          else make_p<EMU>(hi, cs, m_ref, pk, sum0, sum1);
+          make_p<EMU>(hi, cs, m_ref, pk, sum0, sum1);
           tmem_st32(tS + 32, pk);  // keys 64..127 -> columns 32..63
           tmem_wait_st();
           tc_fence_before_sync();

@@ -11,17 +11,47 @@
 // kernel rotates the tree's queries and keys, so that the attention kernels read them as
 // if the caller had done it. Results are rounded to bf16 like the caller's tensors.
 //
-// One CTA per (sequence, node slot); nodes past a sequence's tree do nothing. The
-// depth walk follows parent links through shared memory and stops at the root or at
-// the first link that is not a rooted tree's (the attention kernel reports that tree).
-// The angle is reduced modulo 2 pi in double precision and its sine and cosine taken in
-// float, so that large positions (10^5 and more) keep their precision.
+// One CTA per (sequence, node slot); nodes past a sequence's tree do nothing. The CTA
+// first issues the loads of its node's q and k_tree rows (they do not depend on the
+// position), then finds the depth: every thread takes one node of the sequence and the
+// parent links are followed by pointer jumping in shared memory (after round r each
+// node knows its ancestor 2^r levels up and its distance to it, so seven rounds cover
+// 128 levels); a link that is not a rooted tree's stops the jumping there (the attention
+// kernel reports that tree). The angle is reduced modulo 2 pi in double precision and
+// its sine and cosine taken in float, so that large positions (10^5 and more) keep their
+// precision.
 #include "ls_device.cuh"
 
 namespace ls {
 namespace {
 
-constexpr int kRopeThreads = 128;
+constexpr int kRopeThreads = 256;
+constexpr int kPrefetch = 2;  // (head, 8-pair group) items per thread loaded up front
+
+__device__ __forceinline__ void rotate8(const uint4& lo, const uint4& hi, const float* cos_s, const float* sin_s,
+                                        int e0, uint4& olo, uint4& ohi) {
+  const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w}, hw[4] = {hi.x, hi.y, hi.z, hi.w};
+  uint32_t ol[4], oh[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t rl = 0u, rh = 0u;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = e0 + 2 * w + k;
+      const float x1 = bf16_to_f32((uint16_t)(lw[w] >> (16 * k)));
+      const float x2 = bf16_to_f32((uint16_t)(hw[w] >> (16 * k)));
+      const float c = cos_s[e], s = sin_s[e];
+      const float y1 = fmaf(x1, c, -x2 * s);  // first of the pair
+      const float y2 = fmaf(x2, c, x1 * s);   // second of the pair
+      rl |= (uint32_t)f32_to_bf16(y1) << (16 * k);
+      rh |= (uint32_t)f32_to_bf16(y2) << (16 * k);
+    }
+    ol[w] = rl;
+    oh[w] = rh;
+  }
+  olo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+  ohi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+}
 
 __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a) {
   const Plan& p = a.p;
@@ -32,27 +62,51 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
   int base = 0, n = 0;
   tree_range(p, a.cu_tree, b, &base, &n);
   if (i >= n) return;
-
-  __shared__ int32_t par[kMaxTree];
-  __shared__ float cos_s[64], sin_s[64];
-  __shared__ int32_t depth_s;
   const int tid = threadIdx.x;
-  for (int x = tid; x < n; x += kRopeThreads) par[x] = a.parent[(size_t)base + x];
-  __syncthreads();
-  if (tid == 0) {
-    int x = i, depth = 0;
-    for (int step = 0; step < n && x > 0; ++step) {
-      const int pp = par[x];
-      if (pp < 0 || pp >= x) break;  // not a rooted tree: the attention kernel reports it
-      x = pp;
-      ++depth;
+  const int half = p.d / 2;
+  const int groups = half / 8;  // items: (head, group of 8 pairs); q heads first, then k_tree's
+  const int items = (p.Hq + p.Hkv) * groups;
+  const size_t node = (size_t)base + i;
+  auto src_of = [&](int it) -> const uint16_t* {
+    const int hh = it / groups, e0 = (it % groups) * 8;
+    return hh < p.Hq ? a.q + (node * p.Hq + hh) * p.d + e0 : a.k_tree + (node * p.Hkv + (hh - p.Hq)) * p.d + e0;
+  };
+  auto dst_of = [&](int it) -> uint16_t* {
+    const int hh = it / groups, e0 = (it % groups) * 8;
+    return hh < p.Hq ? a.q_rot + (node * p.Hq + hh) * p.d + e0 : a.k_rot + (node * p.Hkv + (hh - p.Hq)) * p.d + e0;
+  };
+  uint4 lo[kPrefetch], hi[kPrefetch];
+#pragma unroll
+  for (int k = 0; k < kPrefetch; ++k) {
+    const int it = tid + k * kRopeThreads;
+    if (it < items) {
+      lo[k] = *reinterpret_cast<const uint4*>(src_of(it));
+      hi[k] = *reinterpret_cast<const uint4*>(src_of(it) + half);
     }
-    depth_s = depth;
+  }
+
+  __shared__ int32_t anc[2][kMaxTree], dist[2][kMaxTree];
+  __shared__ float cos_s[64], sin_s[64];
+  if (tid < n) {
+    const int32_t pp = a.parent[(size_t)base + tid];
+    const bool link = tid > 0 && pp >= 0 && pp < tid;  // a valid link one level up
+    anc[0][tid] = link ? pp : tid;                     // the root (or a bad link) points at itself
+    dist[0][tid] = link ? 1 : 0;
   }
   __syncthreads();
+  int cur = 0;
+  for (int r = 0; r < 7; ++r) {  // 2^7 = 128 >= any depth
+    if (tid < n) {
+      const int up = anc[cur][tid];
+      anc[cur ^ 1][tid] = anc[cur][up];
+      dist[cur ^ 1][tid] = dist[cur][tid] + (up != tid ? dist[cur][up] : 0);
+    }
+    cur ^= 1;
+    __syncthreads();
+  }
+  const int depth = dist[cur][i];
   const int32_t L = max(a.cu[b + 1] - a.cu[b], 0);
-  const double pos = (double)L + (double)depth_s;
-  const int half = p.d / 2;
+  const double pos = (double)L + (double)depth;
   if (tid < half) {
     // theta_e = base^(-2e/d); the angle pos * theta_e reduced to [-pi, pi]
     const double inv_freq = exp2(-(2.0 * tid / p.d) * a.log2_theta);
@@ -68,44 +122,23 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
   }
   __syncthreads();
 
-  // items: (head, group of 8 pairs); q heads first, then the kv heads of k_tree
-  const int groups = half / 8;
-  const int items = (p.Hq + p.Hkv) * groups;
-  const size_t node = (size_t)base + i;
-  for (int it = tid; it < items; it += kRopeThreads) {
-    const int hh = it / groups, e0 = (it % groups) * 8;
-    const uint16_t* src;
-    uint16_t* dst;
-    if (hh < p.Hq) {
-      src = a.q + (node * p.Hq + hh) * p.d;
-      dst = a.q_rot + (node * p.Hq + hh) * p.d;
-    } else {
-      src = a.k_tree + (node * p.Hkv + (hh - p.Hq)) * p.d;
-      dst = a.k_rot + (node * p.Hkv + (hh - p.Hq)) * p.d;
-    }
-    const uint4 lo = *reinterpret_cast<const uint4*>(src + e0);
-    const uint4 hi = *reinterpret_cast<const uint4*>(src + e0 + half);
-    const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w}, hw[4] = {hi.x, hi.y, hi.z, hi.w};
-    uint32_t ol[4], oh[4];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t rl = 0u, rh = 0u;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int e = e0 + 2 * w + k;
-        const float x1 = bf16_to_f32((uint16_t)(lw[w] >> (16 * k)));
-        const float x2 = bf16_to_f32((uint16_t)(hw[w] >> (16 * k)));
-        const float c = cos_s[e], s = sin_s[e];
-        const float y1 = fmaf(x1, c, -x2 * s);  // first of the pair
-        const float y2 = fmaf(x2, c, x1 * s);   // second of the pair
-        rl |= (uint32_t)f32_to_bf16(y1) << (16 * k);
-        rh |= (uint32_t)f32_to_bf16(y2) << (16 * k);
-      }
-      ol[w] = rl;
-      oh[w] = rh;
+  for (int k = 0; k < kPrefetch; ++k) {
+    const int it = tid + k * kRopeThreads;
+    if (it < items) {
+      uint4 olo, ohi;
+      rotate8(lo[k], hi[k], cos_s, sin_s, (it % groups) * 8, olo, ohi);
+      *reinterpret_cast<uint4*>(dst_of(it)) = olo;
+      *reinterpret_cast<uint4*>(dst_of(it) + half) = ohi;
     }
-    *reinterpret_cast<uint4*>(dst + e0) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-    *reinterpret_cast<uint4*>(dst + e0 + half) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+  }
+  for (int it = tid + kPrefetch * kRopeThreads; it < items; it += kRopeThreads) {  // large head counts
+    const uint4 l1 = *reinterpret_cast<const uint4*>(src_of(it));
+    const uint4 h1 = *reinterpret_cast<const uint4*>(src_of(it) + half);
+    uint4 olo, ohi;
+    rotate8(l1, h1, cos_s, sin_s, (it % groups) * 8, olo, ohi);
+    *reinterpret_cast<uint4*>(dst_of(it)) = olo;
+    *reinterpret_cast<uint4*>(dst_of(it) + half) = ohi;
   }
 }
 
