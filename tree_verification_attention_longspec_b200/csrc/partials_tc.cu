@@ -277,16 +277,20 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
-    // Ring order = consumption order: K(0), V(0), K(1), V(1), ...
-    if (lane == 0) {
+    // Ring order = consumption order: K(0), V(0), K(1), V(1), ... The whole warp walks the
+    // blocks; lane 0 arms the barriers and issues whole-block boxes, and for a paged cache
+    // the lanes issue the block's page boxes (and read their page-table entries) at once.
+    {
       // Q: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows past the
       // batch's last node read as zeros)
       auto load_q = [&]() {
-        mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
 #pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
-                      tree_base + tok0);
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
+                        tree_base + tok0);
+        }
       };
       // When the tree kernel writes q and k_tree (rotated), this grid may start before
       // that grid ends: the prefix loads go ahead, Q and the tree block wait for it.
@@ -302,6 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         load_q();
         q_loaded = true;
       }
+      // a page box is bh rows (the page, or 128 rows of a larger page); lane l issues box
+      // l / kPanels, panel l % kPanels
+      const int bh = paged ? (a.page_size < kBlockN ? a.page_size : kBlockN) : kBlockN;
+      const int n_boxes = (kBlockN / bh) * C::kPanels;
+      const int n_pages = paged ? (seq_len + a.page_size - 1) / a.page_size : 0;
       int issued = 0, slot = 0, use = 0;
       bool ok = true;
       for (int j = 0; j < nbt && ok; ++j) {
@@ -315,35 +324,35 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           wait_prior();
         }
         const bool pieces = paged && !tree;  // the block's rows come page by page
+        // this lane's page box of the block: a page-table entry is only a TMA coordinate,
+        // so a bad one reads zeros or another page, never outside the cache; boxes past
+        // the sequence end read its last page (masked)
+        int prow = 0;
+        const int pc = lane / C::kPanels, pn_l = lane % C::kPanels;
+        if (pieces && lane < n_boxes) {
+          const int key = c.key_skip + c.key_begin + j * kBlockN + pc * bh;
+          int lp = key / a.page_size;
+          if (lp >= n_pages) lp = n_pages - 1;
+          if (lp >= a.max_pages) lp = a.max_pages - 1;
+          prow = a.page_table[(size_t)c.b * a.max_pages + lp] * a.page_size + key % a.page_size;
+        }
         for (int kv = 0; kv < 2; ++kv) {
-          if (!mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs)) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs))) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bars->full[slot], C::kTileBytes);
+          if (lane == 0) mbar_arrive_expect_tx(&bars->full[slot], C::kTileBytes);
+          __syncwarp();
           uint8_t* dst = smem + C::kSlotOff + slot * C::kTileBytes;
           const CUtensorMap* map = tree ? (kv ? &P.tmap_vt : &P.tmap_kt) : (kv ? &P.tmap_v : &P.tmap_k);
           if (!pieces) {
-#pragma unroll
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
-          } else {
-            // boxes of bh rows (the page, or 128 rows of a larger page); pieces past the
-            // sequence end read its last page (masked). A page-table entry is only a TMA
-            // coordinate, so a bad one reads zeros or another page, never outside the cache.
-            const int bh = a.page_size < kBlockN ? a.page_size : kBlockN;
-            const int n_pages = (seq_len + a.page_size - 1) / a.page_size;
-            for (int pc = 0; pc < kBlockN / bh; ++pc) {
-              const int key = c.key_skip + c.key_begin + j * kBlockN + pc * bh;
-              int lp = key / a.page_size;
-              if (lp >= n_pages) lp = n_pages - 1;
-              if (lp >= a.max_pages) lp = a.max_pages - 1;
-              const int prow = a.page_table[(size_t)c.b * a.max_pages + lp] * a.page_size + key % a.page_size;
+            if (lane == 0) {
 #pragma unroll
               for (int pn = 0; pn < C::kPanels; ++pn)
-                tma_load_3d(dst + pn * C::kPanelBytes + pc * bh * 128, map, &bars->full[slot], pn * 64, c.kh,
-                            prow);
+                tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
             }
+          } else if (lane < n_boxes) {
+            tma_load_3d(dst + pn_l * C::kPanelBytes + pc * bh * 128, map, &bars->full[slot], pn_l * 64, c.kh, prow);
           }
           ++issued;
           if (++slot == C::kSlots) {
@@ -357,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             load_q();
             q_loaded = true;
           }
-          if (issued == 1 && !mbar_wait_bounded(&bars->full[0], 0, abort, kTimeoutNs)) {
+          if (issued == 1 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[0], 0, abort, kTimeoutNs))) {
             ok = false;
             break;
           }
@@ -365,10 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       }
       // make sure no copy is still writing shared memory when the CTA ends (Q was
       // issued unless the loop stopped before its first load)
-      if (q_loaded) drain_wait(&bars->q_full, 0);
-      const int first = issued > C::kSlots ? issued - C::kSlots : 0;
-      for (int seq = first; seq < issued; ++seq)
-        drain_wait(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1);
+      if (lane == 0) {
+        if (q_loaded) drain_wait(&bars->q_full, 0);
+        const int first = issued > C::kSlots ? issued - C::kSlots : 0;
+        for (int seq = first; seq < issued; ++seq)
+          drain_wait(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1);
+      }
     }
     __syncwarp();
   } else {
