@@ -77,6 +77,7 @@ struct alignas(64) TcParams {
   CUtensorMap tmap_v;
   CUtensorMap tmap_kt;  // tree keys
   CUtensorMap tmap_vt;
+  CUtensorMap tmap_o;   // o_part as [n_chunks * 256 rows][d] fp32, stores of 128 rows x 32 floats
   PartialsArgs a;
 };
 
@@ -261,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     tma_prefetch_map(&P.tmap_q);
     tma_prefetch_map(&P.tmap_k);
     tma_prefetch_map(&P.tmap_v);
+    tma_prefetch_map(&P.tmap_o);
     if (has_tree) {
       tma_prefetch_map(&P.tmap_kt);
       tma_prefetch_map(&P.tmap_vt);
@@ -626,51 +628,40 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       }
       // -------------------------------------------------------------- epilogue
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full[t], 0, abort, kTimeoutNs));
-      // Each warpgroup stages its normalised 128 x D tile in shared memory (16-byte chunk
-      // c of row r at chunk c ^ (r & 7), conflict-free for the per-row writes) and then
-      // writes it out row-contiguously, since the tile's rows are contiguous in o_part.
-      // Tile 0 finishes while tile 1's last PV may still read V from the slot ring, so
-      // it stages over the Q tiles (every QK has completed by o_full[0]); tile 1, last of
-      // all, stages over the ring.
+      // Each warpgroup stages its normalised 128 x D tile in shared memory as D/32 panels
+      // of 128 rows x 128 B, swizzled like the tensor map (16-byte chunk q of row r at
+      // q ^ (r & 7): conflict-free for the per-row writes), and one thread stores the
+      // panels to o_part with TMA. Tile 0 finishes while tile 1's last PV may still read
+      // V from the slot ring, so it stages over the Q tiles (every QK has completed by
+      // o_full[0]); tile 1, last of all, stages over the ring. Rows past the unit's last
+      // row are stored too: they stay inside the chunk's 256-row slot, which no one reads.
       const bool ok_all = bar_and(2 + t, 128, ok);
       if (ok_all) {
         tc_fence_after_sync();
-        constexpr int kChunks = D / 4;  // float4 chunks per row
-        float* stage = reinterpret_cast<float*>(smem + (t == 0 ? C::kQOff : C::kSlotOff));
+        constexpr int kOPanels = D / 32;  // 128-byte panels of an fp32 row
+        uint8_t* stage = smem + (t == 0 ? C::kQOff : C::kSlotOff);
         const float inv = 1.f / l;
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < D / 32; ++q) {  // panel q = columns [32 q, 32 q + 32)
           uint32_t r[32];
           tmem_ld32(tO + 32 * q, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int ch = 8 * q + e;
-            *reinterpret_cast<float4*>(stage + row * D + ((ch ^ (row & 7)) << 2)) =
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<float4*>(stage + q * (128 * 128) + row * 128 + ((e ^ (row & 7)) << 4)) =
                 make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
                             __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
-          }
         }
         const int ur = t * 128 + row;  // row of the unit
         if (ur < rows_here) a.lse_part[(size_t)blockIdx.x * kUnitRows + ur] = m + log2f(l);
+        fence_proxy_async_smem();  // the staged tile is read by the TMA unit
         asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
-        const int tile_rows = min(128, max(0, rows_here - t * 128));
-        float* dst = a.o_part + ((size_t)blockIdx.x * kUnitRows + t * 128) * D;
-        const int wt = tid & 127;
-        const int n4 = tile_rows * kChunks;
-        for (int i0 = 0; i0 < n4; i0 += 8 * 128) {
-          float4 v[8];
+        if ((warp & 3) == 0 && lane == 0 && t * 128 < rows_here) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * 128 + wt;
-            const int rr = i / kChunks, ch = i % kChunks;
-            if (i < n4) v[u] = *reinterpret_cast<const float4*>(stage + rr * D + ((ch ^ (rr & 7)) << 2));
-          }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * 128 + wt;
-            if (i < n4) *reinterpret_cast<float4*>(dst + (size_t)i * 4) = v[u];
-          }
+          for (int q = 0; q < kOPanels; ++q)
+            tma_store_2d(&P.tmap_o, stage + q * (128 * 128), 32 * q, (int)blockIdx.x * kUnitRows + t * 128);
+          bulk_commit();
+          bulk_wait_all();  // the shared memory must stay until the TMA has read it
         }
       }
     }
@@ -726,6 +717,21 @@ bool make_q_map(CUtensorMap* map, const void* base, int D, const Plan& p) {
   return r == CUDA_SUCCESS;
 }
 
+// o_part viewed as [n_chunks * 256 rows][D] fp32; boxes of 128 rows x 32 floats (128 B),
+// 128B-swizzled like the kernel's staging.
+bool make_o_map(CUtensorMap* map, float* base, int D, int64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int EMU>
 cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream) {
   TcParams P;
@@ -736,7 +742,8 @@ cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream
   if (!make_q_map(&P.tmap_q, a.q, D, a.p) || !make_kv_map(&P.tmap_k, a.k_cache, D, a.p.Hkv, kv_rows, box_rows) ||
       !make_kv_map(&P.tmap_v, a.v_cache, D, a.p.Hkv, kv_rows, box_rows) ||
       !make_kv_map(&P.tmap_kt, a.k_tree, D, a.p.Hkv, tree_rows) ||
-      !make_kv_map(&P.tmap_vt, a.v_tree, D, a.p.Hkv, tree_rows))
+      !make_kv_map(&P.tmap_vt, a.v_tree, D, a.p.Hkv, tree_rows) ||
+      !make_o_map(&P.tmap_o, a.o_part, D, (int64_t)a.p.n_chunks * kUnitRows))
     return cudaErrorInvalidValue;
   const int smem = kSmemWindow;
   // opt in to the large shared-memory carve-out once per device
