@@ -99,12 +99,17 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_
   q.N = tree != nullptr && tree->cu_tree != nullptr ? tree->total_nodes : q.B * q.T;
   q.rope = with_tree && tree != nullptr && tree->rope_theta > 0.0 ? 1 : 0;
   q.window = with_tree && tree != nullptr ? tree->window : 0;
+  q.alt = q.T * q.g <= 128 ? 1 : 0;
   if (q.g > ls::kUnitRows) return LS_ERR_UNSUPPORTED;
   q.tpu = ls::kUnitRows / q.g;
   q.rg = ls::ceil_div(q.T, q.tpu);
   q.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)q.d);
   q.scale_log2 = (float)((double)q.scale * 1.4426950408889634074);
-  q.n_combine = (int32_t)(((long long)q.B * q.T * q.Hq + ls::kMergeRows - 1) / ls::kMergeRows);
+  // few output rows (a draft query or a small tree): one row per combine CTA, whose warps
+  // split the row's partials, so that more warps share the merge
+  const long long out_rows = (long long)q.B * q.T * q.Hq;
+  q.combine_wide = out_rows < 4LL * sms ? 1 : 0;
+  q.n_combine = (int32_t)(q.combine_wide ? out_rows : (out_rows + ls::kMergeRows - 1) / ls::kMergeRows);
 
   std::vector<int32_t> blocks(q.B);
   int32_t max_blocks = 0;

@@ -20,7 +20,7 @@ namespace {
 
 constexpr int kPrefetch = 20;  // partials in flight per warp (the headline has 18 per row)
 
-template <int D>
+template <int D, bool WIDE>
 __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   constexpr int E = D / 32;  // head-dim elements per lane
   const Plan& p = a.p;
@@ -32,7 +32,8 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   // Everything that does not depend on the partials is done before the wait: the row's
   // sequence, its chunk range (from cu_seqlens, an input) and the length check.
   const int64_t n_rows = (int64_t)p.B * p.T * p.Hq;
-  const int64_t row = (int64_t)blockIdx.x * kMergeRows + warp;
+  constexpr bool wide = WIDE;  // the CTA's warps share one row
+  const int64_t row = wide ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kMergeRows + warp;
   const bool has_row = row < n_rows;
   int n = 0, cbase = 0, rl = 0;
   int64_t out_row = 0;
@@ -61,26 +62,35 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   // the partials kernel may still be running: wait for its grid to finish
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  if (writes) {
-    float acc[E];
+  float acc[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    float M = -INFINITY, Lsum = 0.f;  // running max of the lse and sum of weights 2^(l - M)
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float M = -INFINITY, Lsum = 0.f;  // running max of the lse and sum of weights 2^(l - M)
+  if (writes) {
     if (lengths_ok) {
-      for (int x0 = 0; x0 < n; x0 += kPrefetch) {
-        const int nx = min(kPrefetch, n - x0);
-        // every lane one chunk's lse and status; up to kPrefetch chunk outputs in flight
+      // the row's partials: one per chunk, or two (rows rl and rl + 128 of the chunk's
+      // slot) when the partials kernel's tiles alternated key blocks
+      const int sh = p.alt ? 1 : 0;
+      const int n_parts = n << sh;
+      const size_t row0 = (size_t)cbase * kUnitRows + rl;
+      auto part_row = [&](int k) -> size_t {  // row of partial k in o_part / lse_part
+        return row0 + (uint32_t)((k >> sh) * kUnitRows + ((k & sh) << 7));
+      };
+      // a wide CTA's warp w takes the batches w, w + 4, ...
+      const int first_batch = wide ? warp * kPrefetch : 0, stride = wide ? kMergeRows * kPrefetch : kPrefetch;
+      for (int x0 = first_batch; x0 < n_parts; x0 += stride) {
+        const int nx = min(kPrefetch, n_parts - x0);
+        // every lane one partial's lse and status; up to kPrefetch outputs in flight
         float lx = -INFINITY;
         if (lane < nx) {
-          lx = a.lse_part[(size_t)(cbase + x0 + lane) * kUnitRows + rl];
-          err |= a.chunk_status[cbase + x0 + lane];
+          lx = a.lse_part[part_row(x0 + lane)];
+          err |= a.chunk_status[cbase + ((x0 + lane) >> sh)];
         }
         float ov[kPrefetch][E];
-        const float* base = a.o_part + ((size_t)(cbase + x0) * kUnitRows + rl) * D + lane * E;
 #pragma unroll
         for (int x = 0; x < kPrefetch; ++x) {
           if (x < nx) {
-            const float* op = base + (size_t)x * kUnitRows * D;
+            const float* op = a.o_part + part_row(x0 + x) * D + lane * E;
             if constexpr (E == 4) {
               const float4 v = *reinterpret_cast<const float4*>(op);
               ov[x][0] = v.x;
@@ -107,7 +117,7 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
 #pragma unroll
         for (int x = 0; x < kPrefetch; ++x) {
           const float w = __shfl_sync(0xffffffffu, wl, x);
-          if (x < nx && w > 0.f) {  // an empty chunk leaves its output slot unwritten
+          if (x < nx && w > 0.f) {  // an empty partial has weight 0 (its output slot is not read)
 #pragma unroll
             for (int e = 0; e < E; ++e) acc[e] = fmaf(w, ov[x][e], acc[e]);
           }
@@ -116,6 +126,36 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
     } else {
       err |= kErrLengths;
     }
+  }
+  if constexpr (WIDE) {
+    // the warps' merges of their batches, joined by warp 0 in the same way (only the wide
+    // instance holds this scratch: a narrow CTA keeps fitting beside a partials CTA)
+    __shared__ float w_m[kMergeRows], w_l[kMergeRows], w_acc[kMergeRows][D];
+    if (lane == 0) {
+      w_m[warp] = M;
+      w_l[warp] = Lsum;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) w_acc[warp][lane * E + e] = acc[e];
+    __syncthreads();
+    if (warp == 0) {
+      float Mt = -INFINITY;
+      for (int w = 0; w < kMergeRows; ++w)
+        if (w_l[w] > 0.f) Mt = fmaxf(Mt, w_m[w]);
+      Lsum = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      for (int w = 0; w < kMergeRows; ++w) {
+        if (!(w_l[w] > 0.f)) continue;  // a warp without partials
+        const float f = exp2f(w_m[w] - Mt);
+        Lsum = fmaf(w_l[w], f, Lsum);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(w_acc[w][lane * E + e], f, acc[e]);
+      }
+      M = Mt;
+    }
+  }
+  if (writes && (!wide || warp == 0)) {
     const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     uint16_t* dst = a.out + out_row * D + lane * E;
 #pragma unroll
@@ -132,7 +172,7 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
   if (threadIdx.x == 0) a.status[blockIdx.x] = err_s;
 }
 
-template <int D>
+template <int D, bool WIDE>
 cudaError_t launch_d(const CombineArgs& a, cudaStream_t stream) {
   // a programmatic dependent of the partials kernel: its CTAs may be scheduled while
   // that grid runs and wait in griddepcontrol.wait
@@ -146,14 +186,15 @@ cudaError_t launch_d(const CombineArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.after_partials ? 1 : 0;  // else an ordinary launch (it reads cu before its wait)
-  return cudaLaunchKernelEx(&cfg, combine_kernel<D>, a);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<D, WIDE>, a);
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
   if (a.p.n_combine == 0) return cudaSuccess;
-  return a.p.d == 64 ? launch_d<64>(a, stream) : launch_d<128>(a, stream);
+  if (a.p.combine_wide) return a.p.d == 64 ? launch_d<64, true>(a, stream) : launch_d<128, true>(a, stream);
+  return a.p.d == 64 ? launch_d<64, false>(a, stream) : launch_d<128, false>(a, stream);
 }
 
 }  // namespace ls

@@ -39,6 +39,8 @@ struct Plan {
   int32_t N;           // tree nodes of the batch: B * T, or cu_tree[B]
   int32_t rope;        // 1: q and k_tree are rotated (RoPE) by the tree kernel first
   int32_t window;      // > 0: sliding window of this many positions; 0: the whole prefix
+  int32_t alt;         // 1: T*g <= 128 rows; the two query tiles take the same rows and
+                       //    alternate key blocks, leaving two partials per chunk
   int32_t rows;        // T * g query rows per (sequence, kv head)
   int32_t tpu;         // tree nodes per unit: floor(kUnitRows / g)
   int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
@@ -46,7 +48,8 @@ struct Plan {
   int32_t with_tree;   // 1: every key list ends with the tree block; 0: prefix keys only
   int32_t uniform_n;   // >= 0: chunks per unit for every sequence; -1: from L_b
   int32_t n_chunks;    // partials-kernel CTAs
-  int32_t n_combine;   // combine CTAs = ceil(B * T * Hq / kMergeRows)
+  int32_t n_combine;   // combine CTAs = ceil(B * T * Hq / kMergeRows), or B * T * Hq when wide
+  int32_t combine_wide;  // 1: one output row per combine CTA, its warps splitting the row's partials
   float scale;         // softmax scale
   float scale_log2;    // softmax scale * log2(e)
 };

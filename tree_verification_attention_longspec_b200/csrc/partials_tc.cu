@@ -20,6 +20,13 @@
 // unit (MUFU), which bounds the softmax, is shared by two warpgroups that are out of
 // phase. Every K/V tile staged in shared memory serves both query tiles.
 //
+// Alternate blocks. When a kv head has at most 128 query rows (T*g <= 128: a small tree,
+// a single draft query), the second tile would hold only padding. Both tiles then take
+// the same rows and alternate key blocks: tile 0 the even blocks of the chunk, tile 1 the
+// odd ones, each with its own S, O and running max, so two chains advance through one
+// key range; their results are two partials of the chunk (rows 0..127 and 128..255 of
+// its slot), merged by the combine like any other.
+//
 // Warp roles (320 threads, one CTA per SM):
 //   warps 0-3  softmax of tile 0, warps 4-7 of tile 1: one thread per query row (= TMEM
 //              lane) holding the block's 128 scores. P is computed against the running
@@ -231,8 +238,11 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
     return;
   }
-  if (nbt == 0) {  // empty key range: an empty partial
-    for (int r = tid; r < rows_here; r += kThreads) a.lse_part[(size_t)blockIdx.x * kUnitRows + r] = -INFINITY;
+  if (nbt == 0) {  // empty key range: an empty partial (two of them when the tiles alternate)
+    for (int r = tid; r < rows_here; r += kThreads) {
+      a.lse_part[(size_t)blockIdx.x * kUnitRows + r] = -INFINITY;
+      if (p.alt) a.lse_part[(size_t)blockIdx.x * kUnitRows + 128 + r] = -INFINITY;
+    }
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
     return;
   }
@@ -315,7 +325,26 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const int n_pages = paged ? (seq_len + a.page_size - 1) / a.page_size : 0;
       int issued = 0, slot = 0, use = 0;
       bool ok = true;
-      for (int j = 0; j < nbt && ok; ++j) {
+      // the MMA thread's order: K(j), V(j) for j = 0, 1, ...; with alternate blocks K(0),
+      // K(1), then V(j) and K(j + 2) for j = 0, 1, ... (no K past the last block)
+      const int n_loads = 2 * nbt;
+      const int pro = nbt < 2 ? nbt : 2, pairs = nbt > 2 ? nbt - 2 : 0;
+      for (int ld = 0; ld < n_loads && ok; ++ld) {
+        int j, kv;
+        if (!p.alt) {
+          j = ld >> 1;
+          kv = ld & 1;
+        } else if (ld < pro) {
+          j = ld;
+          kv = 0;
+        } else if (ld - pro < 2 * pairs) {
+          const int r = ld - pro;
+          j = (r >> 1) + ((r & 1) ? 2 : 0);
+          kv = (r & 1) ? 0 : 1;
+        } else {
+          j = pairs + (ld - pro - 2 * pairs);
+          kv = 1;
+        }
         // prefix block j, or the tree block: the sequence's nodes (the rows after them
         // belong to the next sequence or lie past the tensor, read as zeros; masked)
         const bool tree = j == nb;
@@ -338,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           if (lp >= a.max_pages) lp = a.max_pages - 1;
           prow = a.page_table[(size_t)c.b * a.max_pages + lp] * a.page_size + key % a.page_size;
         }
-        for (int kv = 0; kv < 2; ++kv) {
+        {
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs))) {
             ok = false;
             break;
@@ -425,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         constexpr uint32_t kTile16 = C::kTileBytes >> 4, kPanel16 = C::kPanelBytes >> 4;
         // S_t = Q_t K^T into tile t's score buffer; K sits in ring slot `slot`
         auto issue_qk = [&](int t, int slot) {
-          const uint64_t dq = dq0 + (uint64_t)(t * kQTile16);
+          const uint64_t dq = dq0 + (uint64_t)((p.alt ? 0 : t) * kQTile16);  // both tiles read tile 0's Q rows when alternating
           const uint64_t dk = dk0 + (uint64_t)(slot * kTile16);
           const uint32_t tS = tbase + C::kColS + t * kBlockN;
 #pragma unroll
@@ -459,14 +488,51 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             use ^= 1;
           }
         };
-        bool ok = wait(&bars->q_full, 0) && wait(&bars->full[slot], use);  // Q, K(0)
-        if (ok) {
-          issue_qk(0, slot);
-          issue_qk(1, slot);
-          umma_commit(&bars->empty[slot]);
-          advance();
+        bool ok = wait(&bars->q_full, 0);
+        if (p.alt) {
+          // alternate blocks: tile t takes blocks t, t + 2, ...; S_t = Q K(t)^T first, then
+          // for j = 0, 1, ...: PV of block j for tile j % 2 and that tile's next QK^T
+          for (int t = 0; t < kTiles && t < nbt && ok; ++t) {
+            ok = wait(&bars->full[slot], use);
+            if (!ok) break;
+            issue_qk(t, slot);
+            umma_commit(&bars->empty[slot]);
+            advance();
+          }
+          for (int j = 0; j < nbt && ok; ++j) {
+            const int t = j & 1, i = j >> 1;  // tile and its own block count
+            ok = wait(&bars->full[slot], use);  // V(j)
+            if (!ok) break;
+            const int sv = slot;
+            advance();
+            ok = wait(&bars->p_full[t][0], i & 1);
+            if (!ok) break;
+            issue_pv(t, sv, i, 0);
+            ok = wait(&bars->p_full[t][1], i & 1);
+            if (!ok) break;
+            issue_pv(t, sv, i, 1);
+            umma_commit(&bars->empty[sv]);
+            if (j + 2 < nbt) {
+              ok = wait(&bars->full[slot], use);  // K(j + 2)
+              if (!ok) break;
+              issue_qk(t, slot);
+              umma_commit(&bars->empty[slot]);
+              advance();
+            } else if (t == 0) {
+              umma_commit(&bars->o_full[0]);  // tile 0's last PV; no QK^T follows it
+            }
+          }
         }
-        for (int j = 0; j < nbt && ok; ++j) {
+        if (ok && !p.alt) {
+          ok = wait(&bars->full[slot], use);  // K(0)
+          if (ok) {
+            issue_qk(0, slot);
+            issue_qk(1, slot);
+            umma_commit(&bars->empty[slot]);
+            advance();
+          }
+        }
+        for (int j = 0; j < nbt && ok && !p.alt; ++j) {
           const int sv = slot, uv = use;  // V(j)
           advance();
           const bool more = j + 1 < nbt;
@@ -508,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const uint32_t tO = tbase + lane_base + C::kColO + t * D;
       const float cs = p.scale_log2;
       float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
-      const int ur = t * 128 + row;       // row of the unit
+      const int ur = p.alt ? row : t * 128 + row;  // row of the unit (both tiles' rows when alternating)
       const bool has_row = ur < rows_here;
       const int node = tok0 + ur / p.g;   // its tree node
       int cut = 0;                        // window: first attended key this row sees
@@ -523,8 +589,11 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         cut = window_cut(p, seq_len, depth);
       }
       bool ok = true;
-      for (int j = 0; j < nbt; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], j & 1, abort, kTimeoutNs));
+      // blocks of this tile: all of them, or every other one (from block t) when alternating
+      const int n_mine = p.alt ? (nbt - t + 1) / 2 : nbt;
+      for (int i = 0; i < n_mine; ++i) {
+        const int j = p.alt ? 2 * i + t : i;  // the block
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], i & 1, abort, kTimeoutNs));
         if (!ok) break;
         tc_fence_after_sync();
         int shift = j == nb - 1 ? tail_shift : 0;          // masked leading columns (this row)
@@ -583,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             // this tile issued before S_t(j) has completed (s_full), and PV_t(j) waits for
             // this warpgroup's P. f = 1 where m is unchanged, 0 before the first block.
             const float f = m == m_new ? 1.f : ex2_approx(m - m_new);
-            if (j > 0) {
+            if (i > 0) {
 #pragma unroll
               for (int q = 0; q < D / 16; ++q) {
                 uint32_t o[16];
@@ -652,11 +721,11 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
                 make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
                             __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
-        const int ur = t * 128 + row;  // row of the unit
-        if (ur < rows_here) a.lse_part[(size_t)blockIdx.x * kUnitRows + ur] = m + log2f(l);
+        // this tile's partial: rows [128 t, 128 t + 128) of the chunk's slot
+        if (has_row) a.lse_part[(size_t)blockIdx.x * kUnitRows + t * 128 + row] = m + log2f(l);
         fence_proxy_async_smem();  // the staged tile is read by the TMA unit
         asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
-        if ((warp & 3) == 0 && lane == 0 && t * 128 < rows_here) {
+        if ((warp & 3) == 0 && lane == 0 && (p.alt || t * 128 < rows_here)) {
 #pragma unroll
           for (int q = 0; q < kOPanels; ++q)
             tma_store_2d(&P.tmap_o, stage + q * (128 * 128), 32 * q, (int)blockIdx.x * kUnitRows + t * 128);
