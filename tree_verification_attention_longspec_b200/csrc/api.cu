@@ -136,6 +136,11 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_
     }
   }
   q.C = best_C;
+  q.cu_n = 0;
+  if (d->cu_seqlens_host != nullptr && q.B < ls::kPlanCu) {
+    q.cu_n = q.B + 1;
+    for (int b = 0; b <= q.B; ++b) q.cu_host[b] = d->cu_seqlens_host[b];
+  }
   q.with_tree = with_tree ? 1 : 0;
   if (d->cu_seqlens_host) {
     q.uniform_n = -1;

@@ -21,7 +21,7 @@ namespace {
 constexpr int kPrefetch = 20;  // partials in flight per warp (the headline has 18 per row)
 
 template <int D, bool WIDE>
-__global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
+__global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineArgs a) {
   constexpr int E = D / 32;  // head-dim elements per lane
   const Plan& p = a.p;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -48,12 +48,15 @@ __global__ void __maxnreg__(112) combine_kernel(CombineArgs a) {
     writes = i < tree_n;  // the node exists in sequence b's tree
     out_row = (int64_t)(tree_base + i) * p.Hq + h;
     int first = 0, total = 0;
-    sequence_chunks(p, a.cu, b, &first, &n, &total);
+    const int32_t* cu = plan_cu(p, a.cu);
+    sequence_chunks(p, cu, b, &first, &n, &total);
     const int32_t L = a.cu[b + 1] - a.cu[b];
     // the device lengths must give the chunk grid the host planned (else some keys were
-    // never attended): same chunk count, and a uniform plan long enough for this L
+    // never attended): same chunk count, a uniform plan long enough for this L, and the
+    // very lengths the kernels addressed keys with when they came with the plan
     lengths_ok = L >= 0 && total == p.n_chunks &&
-                 (p.uniform_n < 0 || (int64_t)prefix_blocks(attended_len(p, L)) + p.with_tree <= (int64_t)p.uniform_n * p.C);
+                 (p.uniform_n < 0 || (int64_t)prefix_blocks(attended_len(p, L)) + p.with_tree <= (int64_t)p.uniform_n * p.C) &&
+                 (p.cu_n == 0 || (a.cu[b] == cu[b] && a.cu[b + 1] == cu[b + 1]));
     int32_t u, r;
     unit_row(p, i, j, &u, &r);
     rl = r;

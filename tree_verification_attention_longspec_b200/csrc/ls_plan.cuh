@@ -28,6 +28,7 @@ constexpr int kBlockN = 128;       // keys per block of the prefix loop
 constexpr int kUnitRows = 256;     // query rows per prefix chunk (two 128-row MMA tiles)
 constexpr int kMaxTree = 128;      // largest supported tree (one key block)
 constexpr int kMergeRows = 4;      // output rows per CTA of the combine kernel (a warp each)
+constexpr int kPlanCu = 33;        // host lengths carried in the plan for batches up to 32
 
 // device-side status bits (combined into one LS_ERR_* by ls_verify_attn_check)
 constexpr uint32_t kErrBadTree = 1u;
@@ -52,7 +53,15 @@ struct Plan {
   int32_t combine_wide;  // 1: one output row per combine CTA, its warps splitting the row's partials
   float scale;         // softmax scale
   float scale_log2;    // softmax scale * log2(e)
+  // The host copy of cu_seqlens, when the caller gave one and B < kPlanCu: the kernels
+  // address keys with it (kernel parameters, no memory round trip at start-up); the
+  // combine checks that the device array agrees. cu_n = 0: the device array is used.
+  int32_t cu_n;
+  int32_t cu_host[kPlanCu];
 };
+
+// The offsets the kernels address keys with: the plan's host copy, else the device array.
+LS_HD const int32_t* plan_cu(const Plan& p, const int32_t* cu_dev) { return p.cu_n ? p.cu_host : cu_dev; }
 
 LS_HD int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
 

@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   const Plan& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  const ChunkCoord c = locate_chunk(p, a.cu, blockIdx.x);
+  const int32_t* cu = plan_cu(p, a.cu);  // kernel parameters when the host gave lengths
+  const ChunkCoord c = locate_chunk(p, cu, blockIdx.x);
   if (!c.valid) return;  // more CTAs than the device lengths need: the combine reports it
   const int n_keys = c.key_end - c.key_begin;
   const int nb = (n_keys + kBlockN - 1) / kBlockN;  // prefix blocks
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   const int tail_end = paged ? n_keys - (nb - 1) * kBlockN : kBlockN;
   const bool has_tree = c.has_tree;
   const int nbt = nb + (has_tree ? 1 : 0);  // blocks, the tree block (block nb) last
-  const int seq_len = a.cu[c.b + 1] - a.cu[c.b];
+  const int seq_len = cu[c.b + 1] - cu[c.b];
   // sliding window: a row at depth d sees the attended keys from window_cut(d) on, which
   // is below 2 * 128, so only the chunks that start there cut rows individually
   const bool win_rows = p.window > 0 && nb > 0 && c.key_begin < 2 * kBlockN;
