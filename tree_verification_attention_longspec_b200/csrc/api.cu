@@ -99,7 +99,6 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_
   q.N = tree != nullptr && tree->cu_tree != nullptr ? tree->total_nodes : q.B * q.T;
   q.rope = with_tree && tree != nullptr && tree->rope_theta > 0.0 ? 1 : 0;
   q.window = with_tree && tree != nullptr ? tree->window : 0;
-  q.alt = q.T * q.g <= 128 ? 1 : 0;
   if (q.g > ls::kUnitRows) return LS_ERR_UNSUPPORTED;
   q.tpu = ls::kUnitRows / q.g;
   q.rg = ls::ceil_div(q.T, q.tpu);

@@ -36,6 +36,7 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
   const int64_t row = wide ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * kMergeRows + warp;
   const bool has_row = row < n_rows;
   int n = 0, cbase = 0, rl = 0;
+  bool alt = false;  // the row's unit ran with alternating tiles: two partials per chunk
   int64_t out_row = 0;
   bool lengths_ok = false, writes = false;
   uint32_t err = 0u;
@@ -60,6 +61,7 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
     int32_t u, r;
     unit_row(p, i, j, &u, &r);
     rl = r;
+    alt = unit_alternates(min(p.tpu, tree_n - u * p.tpu) * p.g);
     cbase = first + (kh * p.rg + u) * n;
   }
   // the partials kernel may still be running: wait for its grid to finish
@@ -73,7 +75,7 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
     if (lengths_ok) {
       // the row's partials: one per chunk, or two (rows rl and rl + 128 of the chunk's
       // slot) when the partials kernel's tiles alternated key blocks
-      const int sh = p.alt ? 1 : 0;
+      const int sh = alt ? 1 : 0;
       const int n_parts = n << sh;
       const size_t row0 = (size_t)cbase * kUnitRows + rl;
       auto part_row = [&](int k) -> size_t {  // row of partial k in o_part / lse_part

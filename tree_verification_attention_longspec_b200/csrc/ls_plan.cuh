@@ -40,8 +40,6 @@ struct Plan {
   int32_t N;           // tree nodes of the batch: B * T, or cu_tree[B]
   int32_t rope;        // 1: q and k_tree are rotated (RoPE) by the tree kernel first
   int32_t window;      // > 0: sliding window of this many positions; 0: the whole prefix
-  int32_t alt;         // 1: T*g <= 128 rows; the two query tiles take the same rows and
-                       //    alternate key blocks, leaving two partials per chunk
   int32_t rows;        // T * g query rows per (sequence, kv head)
   int32_t tpu;         // tree nodes per unit: floor(kUnitRows / g)
   int32_t rg;          // units per (sequence, kv head): ceil(T / tpu)
@@ -118,6 +116,11 @@ LS_HD bool tree_range(const Plan& p, const int32_t* cu_tree, int32_t b, int32_t*
   *n = ok ? e - s : 0;
   return ok;
 }
+
+// A unit of at most 128 existing rows is run with both query tiles on its rows, taking
+// alternate key blocks, and leaves two partials per chunk (rows r and r + 128 of the
+// chunk's slot).
+LS_HD bool unit_alternates(int32_t rows_here) { return rows_here <= 128; }
 
 // Unit and row inside the unit of query row (tree node i, head-in-group j).
 LS_HD void unit_row(const Plan& p, int32_t i, int32_t j, int32_t* unit, int32_t* row) {

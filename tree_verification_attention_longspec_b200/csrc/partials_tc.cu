@@ -20,8 +20,8 @@
 // unit (MUFU), which bounds the softmax, is shared by two warpgroups that are out of
 // phase. Every K/V tile staged in shared memory serves both query tiles.
 //
-// Alternate blocks. When a kv head has at most 128 query rows (T*g <= 128: a small tree,
-// a single draft query), the second tile would hold only padding. Both tiles then take
+// Alternate blocks. When a unit has at most 128 query rows (a small tree, a single draft
+// query, the last nodes of a tree), the second tile would hold only padding. Both tiles then take
 // the same rows and alternate key blocks: tile 0 the even blocks of the chunk, tile 1 the
 // odd ones, each with its own S, O and running max, so two chains advance through one
 // key range; their results are two partials of the chunk (rows 0..127 and 128..255 of
@@ -235,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   tree_range(p, a.cu_tree, c.b, &tree_base, &tree_n);
   const int tok0 = c.rgi * p.tpu;                       // first tree node of the unit
   const int rows_here = min(p.tpu, tree_n - tok0) * p.g;  // rows of the unit that exist
+  const bool alt = unit_alternates(rows_here);             // both tiles on these rows
   if (rows_here <= 0) {  // a unit past the sequence's tree: nothing to attend for
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
     return;
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   if (nbt == 0) {  // empty key range: an empty partial (two of them when the tiles alternate)
     for (int r = tid; r < rows_here; r += kThreads) {
       a.lse_part[(size_t)blockIdx.x * kUnitRows + r] = -INFINITY;
-      if (p.alt) a.lse_part[(size_t)blockIdx.x * kUnitRows + 128 + r] = -INFINITY;
+      if (alt) a.lse_part[(size_t)blockIdx.x * kUnitRows + 128 + r] = -INFINITY;
     }
     if (tid == 0) a.chunk_status[blockIdx.x] = 0u;
     return;
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const int pro = nbt < 2 ? nbt : 2, pairs = nbt > 2 ? nbt - 2 : 0;
       for (int ld = 0; ld < n_loads && ok; ++ld) {
         int j, kv;
-        if (!p.alt) {
+        if (!alt) {
           j = ld >> 1;
           kv = ld & 1;
         } else if (ld < pro) {
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         constexpr uint32_t kTile16 = C::kTileBytes >> 4, kPanel16 = C::kPanelBytes >> 4;
         // S_t = Q_t K^T into tile t's score buffer; K sits in ring slot `slot`
         auto issue_qk = [&](int t, int slot) {
-          const uint64_t dq = dq0 + (uint64_t)((p.alt ? 0 : t) * kQTile16);  // both tiles read tile 0's Q rows when alternating
+          const uint64_t dq = dq0 + (uint64_t)((alt ? 0 : t) * kQTile16);  // both tiles read tile 0's Q rows when alternating
           const uint64_t dk = dk0 + (uint64_t)(slot * kTile16);
           const uint32_t tS = tbase + C::kColS + t * kBlockN;
 #pragma unroll
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           }
         };
         bool ok = wait(&bars->q_full, 0);
-        if (p.alt) {
+        if (alt) {
           // alternate blocks: tile t takes blocks t, t + 2, ...; S_t = Q K(t)^T first, then
           // for j = 0, 1, ...: PV of block j for tile j % 2 and that tile's next QK^T
           for (int t = 0; t < kTiles && t < nbt && ok; ++t) {
@@ -524,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             }
           }
         }
-        if (ok && !p.alt) {
+        if (ok && !alt) {
           ok = wait(&bars->full[slot], use);  // K(0)
           if (ok) {
             issue_qk(0, slot);
@@ -533,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             advance();
           }
         }
-        for (int j = 0; j < nbt && ok && !p.alt; ++j) {
+        for (int j = 0; j < nbt && ok && !alt; ++j) {
           const int sv = slot, uv = use;  // V(j)
           advance();
           const bool more = j + 1 < nbt;
@@ -575,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const uint32_t tO = tbase + lane_base + C::kColO + t * D;
       const float cs = p.scale_log2;
       float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
-      const int ur = p.alt ? row : t * 128 + row;  // row of the unit (both tiles' rows when alternating)
+      const int ur = alt ? row : t * 128 + row;  // row of the unit (both tiles' rows when alternating)
       const bool has_row = ur < rows_here;
       const int node = tok0 + ur / p.g;   // its tree node
       int cut = 0;                        // window: first attended key this row sees
@@ -591,9 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       }
       bool ok = true;
       // blocks of this tile: all of them, or every other one (from block t) when alternating
-      const int n_mine = p.alt ? (nbt - t + 1) / 2 : nbt;
+      const int n_mine = alt ? (nbt - t + 1) / 2 : nbt;
       for (int i = 0; i < n_mine; ++i) {
-        const int j = p.alt ? 2 * i + t : i;  // the block
+        const int j = alt ? 2 * i + t : i;  // the block
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], i & 1, abort, kTimeoutNs));
         if (!ok) break;
         tc_fence_after_sync();
@@ -726,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         if (has_row) a.lse_part[(size_t)blockIdx.x * kUnitRows + t * 128 + row] = m + log2f(l);
         fence_proxy_async_smem();  // the staged tile is read by the TMA unit
         asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
-        if ((warp & 3) == 0 && lane == 0 && (p.alt || t * 128 < rows_here)) {
+        if ((warp & 3) == 0 && lane == 0 && (alt || t * 128 < rows_here)) {
 #pragma unroll
           for (int q = 0; q < kOPanels; ++q)
             tma_store_2d(&P.tmap_o, stage + q * (128 * 128), 32 * q, (int)blockIdx.x * kUnitRows + t * 128);
