@@ -92,6 +92,15 @@ def test_paged_small_all_rows(page_size, d):
     _check(inp, o, l_)
 
 
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_paged_two_tile_units_all_rows(page_size):
+    # 192 rows per kv head (g = 8, T = 24): a unit of two 128-row tiles, not alternating
+    w = Workload("paged2t", 3, 16, 2, 128, 24, 0, "bfs", input_scale=1.0, lengths=[777, 3000, 130])
+    inp = make_inputs(w, seed=4)
+    o, l_ = _run_paged(inp, page_size)
+    _check(inp, o, l_)
+
+
 @pytest.mark.parametrize("page_size", [16, 128])
 def test_paged_headline_sampled_rows(page_size):
     inp = make_inputs(WORKLOADS["qwen7b_L64k_T64_h28x4_d128"], seed=0)
