@@ -1,6 +1,6 @@
 """Compile the fp64 oracle (plain C, OpenMP) into oracle/liboracle.so.
 
-Test infrastructure: building the checker is not using it.
+Test infrastructure: compiling the oracle here does not put it on any product path.
 """
 from __future__ import annotations
 
