@@ -83,6 +83,17 @@ def test_edge_cases_all_rows(B, Hq, Hkv, d, T, lengths, tree):
     _compare(inp, out, lse)
 
 
+def test_large_batch_with_host_lengths():
+    # more sequences than the plan carries host lengths for (32): the kernels read the
+    # device cu_seqlens, with per-sequence chunk counts from the host copy
+    rng = np.random.default_rng(9)
+    lengths = [int(x) for x in rng.integers(0, 700, size=40)]
+    inp = _small(40, 8, 2, 64, 6, lengths, "uniform", seed=9)
+    out, lse, st = run_gpu(inp)
+    assert st == 0
+    _compare(inp, out, lse)
+
+
 def test_uniform_plan_without_host_lengths():
     inp = _small(4, 16, 4, 128, 12, [5000, 0, 130, 2049], "uniform", seed=3)
     out, lse, st = run_gpu(inp, host_lengths=False)
