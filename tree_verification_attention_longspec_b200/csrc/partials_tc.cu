@@ -548,6 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             ok = wait(&bars->p_full[t][1], pp);
             if (!ok) break;
             issue_pv(t, sv, j, 1);
+            // V(j) is free once both tiles' PV have read it: released before the next QK^T,
+            // so that its refill (a few microseconds in flight) starts that much earlier
+            if (t == 1) umma_commit(&bars->empty[sv]);
             if (!more && t == 0) umma_commit(&bars->o_full[0]);  // tile 0's epilogue may start
             if (more) {
               if (t == 0) ok = wait(&bars->full[sk], uk);
@@ -556,7 +559,6 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             }
           }
           if (!ok) break;
-          umma_commit(&bars->empty[sv]);
           if (more) {
             umma_commit(&bars->empty[sk]);
             advance();
