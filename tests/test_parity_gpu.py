@@ -83,6 +83,24 @@ def test_edge_cases_all_rows(B, Hq, Hkv, d, T, lengths, tree):
     _compare(inp, out, lse)
 
 
+MULTI_UNIT = [
+    # d = 128 with two or four 256-row units per kv head, each unit above 128 rows (two
+    # tiles, no alternate blocks). B, Hq, Hkv, T, lengths, tree
+    (2, 14, 2, 64, [300, 1000], "window8"),   # g = 7: units of 252 and 196 rows, ragged tails
+    (3, 16, 2, 64, [129, 0, 2049], "bfs"),    # g = 8: two full units; an empty prefix
+    (1, 32, 4, 128, [777], "chain"),          # g = 8, T = 128: four units per kv head
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,lengths,tree", MULTI_UNIT)
+@pytest.mark.parametrize("host_lengths", [True, False])
+def test_multi_unit_kv_heads_all_rows(B, Hq, Hkv, T, lengths, tree, host_lengths):
+    inp = _small(B, Hq, Hkv, 128, T, lengths, tree, seed=B * 11 + T)
+    out, lse, st = run_gpu(inp, host_lengths=host_lengths)
+    assert st == 0
+    _compare(inp, out, lse)
+
+
 def test_large_batch_with_host_lengths():
     # more sequences than the plan carries host lengths for (32): the kernels read the
     # device cu_seqlens, with per-sequence chunk counts from the host copy
