@@ -177,12 +177,32 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- traffic record
+def code_lines(text):
+    """The source's code: each line cut at a `//` comment outside a string literal,
+    trailing blanks removed, empty lines dropped (a comment edit leaves it unchanged)."""
+    out = []
+    for line in text.splitlines():
+        in_str, cut = False, len(line)
+        for i, ch in enumerate(line):
+            if ch == '"' and (i == 0 or line[i - 1] != "\\"):
+                in_str = not in_str
+            elif not in_str and line.startswith("//", i):
+                cut = i
+                break
+        code = line[:cut].rstrip()
+        if code:
+            out.append(code)
+    return "\n".join(out)
+
+
 def kernel_source_hash():
+    """Hash of the CUDA sources' code (comments excluded), which the recorded ncu traffic
+    must match."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(DOMINANT_KERNEL_SRC)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(DOMINANT_KERNEL_SRC, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(DOMINANT_KERNEL_SRC, name), encoding="utf-8") as f:
+                h.update(name.encode() + code_lines(f.read()).encode())
     return h.hexdigest()[:16]
 
 

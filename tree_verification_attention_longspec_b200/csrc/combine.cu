@@ -10,9 +10,10 @@
 // One warp per output row (tree node i of sequence b, query head h); lanes split the
 // head dimension. Rows are enumerated as if every sequence had T nodes; with
 // per-sequence trees (cu_tree) the rows past a sequence's own tree have no output. The kernel is launched as a programmatic dependent of the partials
-// kernel and waits for its results with griddepcontrol.wait. It uses no shared memory
-// beyond a status word, so one of its CTAs fits beside a partials CTA on an SM and is
-// ready when that grid ends.
+// kernel and waits for its results with griddepcontrol.wait: its CTAs are launched onto
+// the SMs the partials grid leaves free (and onto each SM as a partials CTA leaves; the
+// partials CTA's registers keep them apart while it runs), do their row bookkeeping and
+// wait there.
 #include "ls_device.cuh"
 
 namespace ls {
@@ -134,7 +135,7 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
   }
   if constexpr (WIDE) {
     // the warps' merges of their batches, joined by warp 0 in the same way (only the wide
-    // instance holds this scratch: a narrow CTA keeps fitting beside a partials CTA)
+    // instance holds this scratch)
     __shared__ float w_m[kMergeRows], w_l[kMergeRows], w_acc[kMergeRows][D];
     if (lane == 0) {
       w_m[warp] = M;

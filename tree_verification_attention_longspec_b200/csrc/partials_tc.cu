@@ -101,9 +101,8 @@ struct Bars {
   int16_t parent[kMaxTree];   // the sequence's tree (chunks that hold the tree block)
 };
 
-// The kernel asks for the dynamic window of a CTA less 1 KB (so that one CTA of the
-// combine kernel, which needs no shared memory beyond the 1 KB every CTA reserves, can
-// wait beside it) and aligns its layout up to 1024 bytes inside it (the 128-byte
+// The kernel asks for the dynamic window of a CTA less 1 KB and aligns its layout up to
+// 1024 bytes inside it (the 128-byte
 // swizzle atom repeats every 1024 bytes).
 constexpr int kSmemWindow = 232448 - 1024;
 template <int D>
