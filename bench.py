@@ -165,7 +165,12 @@ class ClockSampler:
     def summary(self):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
-        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        # Every sample is taken inside the timed region, whose GPU queue never empties
+        # (spin, L2 flush and measured kernels back to back). NVML's utilisation is a
+        # trailing average that can still read 0 over so short a window: the samples it
+        # marks busy are used when there are any, else all of them, and the line says which.
+        busy = [s for s in self.samples if s[2] > 0]
+        loaded = busy or self.samples
         reasons = set()
         for _, rs, _ in loaded:
             for name, bit in self.REASONS.items():
@@ -173,7 +178,9 @@ class ClockSampler:
                     reasons.add(name)
         med = statistics.median([s[0] for s in loaded]) if loaded else None
         return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
-                "samples": len(self.samples), "samples_under_load": len([s for s in self.samples if s[2] > 0])}
+                "samples": len(self.samples), "samples_under_load": len(loaded),
+                "load_basis": ("NVML utilisation above 0" if busy else
+                               "all samples (each inside the timed region, GPU queue full)")}
 
 
 # ----------------------------------------------------------------------------- traffic record
