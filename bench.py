@@ -297,6 +297,86 @@ def run_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- other configs
+CONFIG_WORKLOADS = ("tiny_L1k_T16_h4x1_d64", "llama8b_L16k_T64_h32x8_d128", "70b_L128k_T128_h64x8_d128_bfs",
+                    "ragged_b8_L4k-32k_T64_h32x8_d128")
+
+
+def roofline_of(fig, part_s, step_s, peaks):
+    """Kernel and step roofline fractions of one workload against the measured peaks."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    t_bytes = fig["partials_bytes"] / (hbm * 1e9)
+    t_flops = fig["partials_flops"] / (tc * 1e12)
+    bound = "tensor" if t_flops >= t_bytes else "hbm"
+    roof_step = max(fig["step_bytes"] / (hbm * 1e9), fig["step_flops"] / (tc * 1e12))
+    return {"bound": bound, "kernel_frac": max(t_flops, t_bytes) / part_s, "step_frac": roof_step / step_s,
+            "roofline_us": roof_step * 1e6}
+
+
+def time_config(name, steps, warmup, spin_cycles, flush, dev, peaks):
+    """One BASELINE config timed like the headline (L2 flushed and the step queued before
+    each call): whole ls_verify_attn call and the partials kernel alone, µs per call."""
+    import torch
+
+    from tree_verification_attention_longspec_b200 import binding
+    w = WORKLOADS[name]
+    inp = make_inputs(w, seed=0)
+    fig = workload_figures(inp)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    d_in = dict(q=bf(inp.q), k_cache=bf(inp.k_cache), v_cache=bf(inp.v_cache), k_tree=bf(inp.k_tree),
+                v_tree=bf(inp.v_tree),
+                parent=torch.from_numpy(np.ascontiguousarray(inp.parent, dtype=np.int32)).to(dev),
+                cu=torch.from_numpy(np.ascontiguousarray(inp.cu_seqlens, dtype=np.int32)).to(dev))
+    op = binding.VerifyAttn(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.tree_size,
+                            cu_seqlens_host=inp.cu_seqlens, device=dev)
+    out = torch.empty_like(d_in["q"])
+    lse = torch.empty(out.shape[0], w.num_q_heads, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    ptr = {k: v.data_ptr() for k, v in d_in.items()}
+    dims, ws, wsb = op.dims, op.workspace.data_ptr(), op.ws_bytes
+
+    def full_call():
+        rc = binding.call_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["k_tree"], ptr["v_tree"],
+                              ptr["parent"], ptr["cu"], out.data_ptr(), lse.data_ptr(), dims, ws, wsb, sp)
+        if rc:
+            raise binding.LSError(rc, "ls_verify_attn")
+
+    def partials():
+        rc = binding.call_partials_raw(ptr["q"], ptr["k_cache"], ptr["v_cache"], ptr["k_tree"], ptr["v_tree"],
+                                       ptr["parent"], ptr["cu"], dims, ws, wsb, sp)
+        if rc:
+            raise binding.LSError(rc, "ls_verify_attn_partials")
+
+    for _ in range(warmup):
+        flush.zero_()
+        full_call()
+    torch.cuda.synchronize(dev)
+    times = {}
+    for label, fn in (("call", full_call), ("partials", partials)):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for k in range(steps):
+            flush.zero_()
+            torch.cuda._sleep(spin_cycles)
+            ev[k][0].record(stream)
+            fn()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        times[label] = float(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    st = op.check()
+    if st != 0:
+        raise binding.LSError(st, f"device status ({name})")
+    call_ms, part_ms = max_over_ranks([times["call"], times["partials"]], device=dev)
+    r = roofline_of(fig, part_ms / 1000.0, call_ms / 1000.0, peaks)
+    return {"us_per_call": call_ms * 1000.0, "partials_us": part_ms * 1000.0, "bound": r["bound"],
+            "kernel_frac": r["kernel_frac"], "step_frac": r["step_frac"], "roofline_us": r["roofline_us"],
+            "kv_hbm_gbs": fig["kv_bytes"] / (call_ms / 1000.0) / 1e9, "steps": steps, "plan": op.plan}
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
@@ -480,6 +560,21 @@ def run_ours(args):
     if st != 0:
         raise binding.LSError(st, "device status after timing")
 
+    # the other BASELINE configs, timed the same way in the same run (fewer steps each)
+    configs = None
+    plain = not (args.cross or args.paged or args.rope > 0 or args.window > 0 or inp.cu_tree is not None)
+    if plain and not args.no_configs and w.name == HEADLINE.name:
+        peaks_c, _ = load_peaks()
+        cfg_sampler = ClockSampler(local)
+        with cfg_sampler:
+            configs = {name: time_config(name, max(3, min(K, args.config_steps)), args.warmup, spin_cycles, flush,
+                                         dev, peaks_c)
+                       for name in CONFIG_WORKLOADS}
+        configs["clocks"] = cfg_sampler.summary()
+        configs["timing"] = ("each config: L2 flushed and the step queued before every call, CUDA events; "
+                             "us_per_call = ls_verify_attn, partials_us = the partials kernel alone; "
+                             "kernel_frac / step_frac against MEASURED_PEAKS.json (bf16 burst, HBM copy)")
+
     # e2e through the public call with host buffers: H2D of every input, the call, D2H of out+lse
     e2e = None
     if not args.no_e2e:
@@ -560,6 +655,8 @@ def run_ours(args):
                               "partials kernel timed in K further partials-only launches after the K "
                               "steps, same L2 flush and queueing"),
             "clocks": sampler.summary(), "e2e": e2e}
+    if configs is not None:
+        line["configs"] = configs
     if world == 1 and not args.no_cpu_baseline:
         us, n, dt, cores = time_oracle(inp, target_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -662,6 +759,10 @@ def main():
     ap.add_argument("--accept", type=int, default=0,
                     help="time greedy tree acceptance with bf16 logits of this vocabulary size instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other BASELINE configs after the headline")
+    ap.add_argument("--config-steps", type=int, default=30,
+                    help="timed calls per other config (at most --steps)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--spin-us", type=float, default=150.0,
                     help="GPU spin before each timed step so the step is queued before it starts")

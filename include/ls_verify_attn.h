@@ -21,10 +21,12 @@
  *   out  = sum_{x in visible(i)} exp(s_x - lse) * v_x[kh,:]
  *
  * All calls are C functions with plain pointers and sizes. Device pointers are CUDA
- * device (or managed) memory of the current device. The library allocates no memory
- * and keeps no state between calls; every buffer, including the workspace, belongs
- * to the caller. Nothing in this library traps or aborts: errors come back as status
- * codes.
+ * device (or managed) memory of the current device. The calls that take a workspace
+ * allocate no memory and keep no state between calls: every buffer, including the
+ * workspace, belongs to the caller. The one exception is ls_verify_attn_static (below),
+ * whose scratch is a fixed array in the library's own device memory that keeps what the
+ * last such call left in it. Nothing in this library traps or aborts: errors come back
+ * as status codes.
  */
 #ifndef LS_VERIFY_ATTN_H
 #define LS_VERIFY_ATTN_H
@@ -51,7 +53,9 @@ enum {
   LS_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
   LS_ERR_BAD_TREE = 5,     /* device found parent[] that is not a rooted tree with parent[i] < i */
   LS_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up (pipeline stalled) */
-  LS_ERR_LENGTHS = 7       /* device cu_seqlens disagrees with cu_seqlens_host / max_prefix_len */
+  LS_ERR_LENGTHS = 7,      /* device cu_seqlens disagrees with cu_seqlens_host / max_prefix_len */
+  LS_ERR_INDEX = 8         /* index-checking build (libls_verify_attn_debug.so) only: a kernel formed
+                              a TMA coordinate or global index outside the tensor it addresses */
 };
 
 /* Problem description, passed by pointer to every call. */
@@ -209,12 +213,24 @@ LS_API int ls_verify_attn_paged(const void* q, const void* k_pages, const void* 
  *   values are rounded to bf16, as a caller's own rotation would leave them, and held in
  *   the workspace; v_tree and the cached keys (rotated when they were written) are read
  *   as they are. rope_theta = 0: q and k_tree are already rotated.
+ *
+ * wait_limit_ns > 0: the longest time (nanoseconds, up to 60 s; more is
+ *   LS_ERR_INVALID_ARG) that any of the partials kernel's device-side waits (a CTA's
+ *   roles hand tiles to one another through shared-memory barriers) may take. A wait
+ *   that runs out stops its CTA: every role lets its copies and tensor-core work in
+ *   flight finish, the CTA frees its tensor memory and returns, and
+ *   ls_verify_attn_check reports LS_ERR_TIMEOUT for the call (its outputs are then
+ *   unspecified; the workspace and the device need no cleaning before the next call).
+ *   It is the stall detector of the pipeline: a healthy call waits microseconds, so
+ *   the default (wait_limit_ns = 0: 4 s) only fires on a stalled GPU. A limit shorter
+ *   than a call's normal waits makes healthy calls fail.
  */
 typedef struct {
   const int32_t* cu_tree;
   int32_t total_nodes;
   int32_t window;
   double rope_theta;
+  uint64_t wait_limit_ns;
 } ls_tree_opts;
 
 /*
@@ -268,7 +284,10 @@ LS_API int ls_cross_attn(const void* q, const void* k_cache, const void* v_cache
  *   - Returns LS_ERR_WORKSPACE if these dims need more than 32 MiB of scratch (see
  *     ls_verify_attn_workspace_size); use ls_verify_attn with a workspace for those.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before capturing any stream.
+ *     (cudaGetSymbolAddress) and keeps it; make that first call before capturing any
+ *     stream. cudaDeviceReset reloads the library's device code, after which the kept
+ *     address may be wrong: a process that resets a device must not call
+ *     ls_verify_attn_static on it again.
  *   - All calls on a device share the one array, which keeps whatever the last call
  *     left in it. Calls whose kernels overlap on the GPU (different streams without an
  *     ordering between them) race on it and give wrong results; order them.
@@ -328,7 +347,8 @@ LS_API int ls_tree_accept_greedy(const void* logits, const int32_t* tree_tokens,
 /*
  * Waits for `stream`, then reads the device-side status that the last ls_verify_attn
  * call with this workspace and these dims recorded. Returns LS_OK, LS_ERR_BAD_TREE,
- * LS_ERR_LENGTHS, LS_ERR_TIMEOUT, or LS_ERR_CUDA if the copy itself failed.
+ * LS_ERR_LENGTHS, LS_ERR_TIMEOUT, LS_ERR_INDEX (index-checking build only), or
+ * LS_ERR_CUDA if the copy itself failed.
  */
 LS_API int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void* stream);
 

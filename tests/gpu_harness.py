@@ -14,11 +14,24 @@ def bf16_ulp(x):
     return np.exp2(np.floor(np.log2(ax)) - 7)
 
 
+WIDEN_AT = 4.0    # |ref| from which half a bf16 ulp (2^-6 = 0.0156) exceeds OUT_ATOL
+
+
 def out_tolerance(ref):
-    """Per-element bound on |out - ref|: 1e-2, except where bf16 itself cannot resolve
-    it. For |ref| >= 2 one bf16 ulp exceeds 2^-7 = 0.0078 and round-to-nearest alone
-    costs half an ulp, so the bound there is one ulp at |ref|."""
-    return np.maximum(OUT_ATOL, bf16_ulp(ref))
+    """Per-element bound on |out - ref|: OUT_ATOL (1e-2) wherever bf16 can meet it.
+
+    `out` is bf16, so rounding the exact result costs up to half a bf16 ulp: 2^-8 at
+    |ref| in [1, 2), 2^-7 = 0.0078 in [2, 4), both below 1e-2; from |ref| = 4 on half an
+    ulp is 2^-6 = 0.0156 and 1e-2 cannot be met. There the bound is half an ulp at |ref|
+    plus the kernel's own error before that rounding. The probabilities P enter the
+    tensor-core PV product as bf16 (relative error 2^-9 each); the kernel normalises by
+    the sum of those rounded weights, so its output is a convex combination of the values
+    whose weights are each off by at most 2 * 2^-9 relative, an error of at most
+    2^-8 * |ref| when the weighted values have the sign of the result (the case for every
+    |ref| >= 4 that a softmax average of the values can reach)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    wide = 0.5 * bf16_ulp(ref) + np.abs(ref) * 2.0 ** -8
+    return np.where(np.abs(ref) >= WIDEN_AT, np.maximum(OUT_ATOL, wide), OUT_ATOL)
 
 
 def to_device(inp, device="cuda:0"):
@@ -59,28 +72,3 @@ def run_gpu(inp, host_lengths=True, scale=0.0, dev=None, op=None):
     o = out.float().cpu().numpy().astype(np.float64).reshape(-1, w.head_dim)
     l = lse.cpu().numpy().astype(np.float64).reshape(-1)
     return o, l, status
-
-
-def sample_rows(inp, n_random=48, seed=0):
-    """Rows r = (b*T+i)*H_q + h covering the first/last node and head of every sequence,
-    the first and last row of every unit (floor(256/g) whole nodes) of every kv head,
-    both ends of every 128-row query tile inside a unit, plus random rows."""
-    w = inp.workload
-    B, T, Hq, Hkv = w.batch, w.tree_size, w.num_q_heads, w.num_kv_heads
-    g = Hq // Hkv
-    tpu = 256 // g
-    rows = set()
-    for b in range(B):
-        for i in (0, T - 1):
-            for h in (0, Hq - 1):
-                rows.add((b * T + i) * Hq + h)
-        for kh in range(Hkv):
-            for n0 in range(0, T, tpu):
-                n_rows = min(tpu, T - n0) * g
-                for rr in (0, 127, 128, n_rows - 1):
-                    if rr < n_rows:
-                        i, j = divmod(rr, g)
-                        rows.add((b * T + n0 + i) * Hq + kh * g + j)
-    rng = np.random.default_rng(seed)
-    rows.update(int(x) for x in rng.integers(0, B * T * Hq, size=n_random))
-    return np.array(sorted(rows), dtype=np.int64)

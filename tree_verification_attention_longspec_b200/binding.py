@@ -15,10 +15,13 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libls_verify_attn.so")
+# the index-checking build of the same sources (tests only): see build.py --debug
+DEBUG_LIB_PATH = os.path.join(_HERE, "lib", "libls_verify_attn_debug.so")
 
 LS_OK = 0
 STATUS_NAMES = {0: "LS_OK", 1: "LS_ERR_INVALID_ARG", 2: "LS_ERR_UNSUPPORTED", 3: "LS_ERR_WORKSPACE",
-                4: "LS_ERR_CUDA", 5: "LS_ERR_BAD_TREE", 6: "LS_ERR_TIMEOUT", 7: "LS_ERR_LENGTHS"}
+                4: "LS_ERR_CUDA", 5: "LS_ERR_BAD_TREE", 6: "LS_ERR_TIMEOUT", 7: "LS_ERR_LENGTHS",
+                8: "LS_ERR_INDEX"}
 EXPORTED = ("ls_verify_attn", "ls_verify_attn_partials", "ls_verify_attn_combine",
             "ls_verify_attn_workspace_size", "ls_verify_attn_check", "ls_status_string",
             "ls_verify_attn_plan", "ls_verify_attn_static", "ls_verify_attn_paged", "ls_cross_attn",
@@ -45,9 +48,10 @@ class PagedKV(ctypes.Structure):
 
 
 class TreeOpts(ctypes.Structure):
-    """ls_tree_opts: per-sequence trees (cu_tree, device address), sliding window, in-kernel RoPE."""
+    """ls_tree_opts: per-sequence trees (cu_tree, device address), sliding window, in-kernel RoPE,
+    and the limit of the kernel's device-side waits (0: the default, 4 s)."""
     _fields_ = [("cu_tree", ctypes.c_void_p), ("total_nodes", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("rope_theta", ctypes.c_double)]
+                ("rope_theta", ctypes.c_double), ("wait_limit_ns", ctypes.c_uint64)]
 
 
 class AcceptDims(ctypes.Structure):
@@ -72,6 +76,17 @@ def load_library(path: str = LIB_PATH):
     global _lib
     if _lib is not None:
         return _lib
+    _lib = _open(path)
+    return _lib
+
+
+def load_debug_library(path: str = DEBUG_LIB_PATH):
+    """Load the index-checking build (a separate library with the same entry points,
+    not the one the other calls here use). Raises if it has not been built."""
+    return _open(path)
+
+
+def _open(path: str):
     if not os.path.exists(path):
         raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m tree_verification_attention_longspec_b200.build`")
@@ -112,7 +127,6 @@ def load_library(path: str = LIB_PATH):
     I = ctypes.POINTER(ctypes.c_int32)
     lib.ls_verify_attn_plan.argtypes = [D, I, I, I]
     lib.ls_verify_attn_plan.restype = ctypes.c_int
-    _lib = lib
     return lib
 
 

@@ -1,10 +1,16 @@
 """Build libls_verify_attn.so (CUDA, sm_100a) in-tree with nvcc.
 
-    python -m tree_verification_attention_longspec_b200.build [--force]
+    python -m tree_verification_attention_longspec_b200.build [--force] [--debug]
 
 Each .cu file under csrc/ is compiled for sm_100a only and the objects are linked
 into one shared library next to this file (lib/), with the CUDA runtime linked
 statically, so the library loads wherever the driver does.
+
+--debug builds the index-checking library, libls_verify_attn_debug.so: the same
+sources compiled with LS_DEBUG, so that every TMA coordinate and global index the
+kernels form is checked against its tensor's extent and a failed check is reported by
+ls_verify_attn_check as LS_ERR_INDEX. It is a separate library with the same entry
+points, for tests; the product library has no checks.
 """
 from __future__ import annotations
 
@@ -21,7 +27,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libls_verify_attn.so")
+LIB_DEBUG = os.path.join(LIBDIR, "libls_verify_attn_debug.so")
 OBJDIR = os.path.join(ROOT, "_build", "obj")
+OBJDIR_DEBUG = os.path.join(ROOT, "_build", "obj_debug")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
@@ -43,23 +51,26 @@ def _headers():
     return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _sources() + _headers() + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, debug: bool = False) -> str:
+    lib, objdir = (LIB_DEBUG, OBJDIR_DEBUG) if debug else (LIB, OBJDIR)
+    if not force and up_to_date(lib):
+        return lib
+    os.makedirs(objdir, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    if debug:
+        extra += ["-DLS_DEBUG"]
 
     def compile_one(src):
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [cc, *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -70,15 +81,15 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
 
     with ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [cc, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-cudart", "static"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
-                ptxas_verbose="--ptxas" in sys.argv))
+                ptxas_verbose="--ptxas" in sys.argv, debug="--debug" in sys.argv))

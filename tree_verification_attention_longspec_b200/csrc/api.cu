@@ -15,6 +15,8 @@ namespace {
 using ls::Plan;
 
 constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitNs = 4000000000ull;  // 4 s
+constexpr uint64_t kMaxWaitNs = 60000000000ull;     // 60 s
 int g_sm_count[kMaxDevices];  // 0 = not queried yet; a benign race writes the same value
 int g_cc_major[kMaxDevices];
 
@@ -71,6 +73,7 @@ int check_tree(const ls_verify_dims* d, const ls_tree_opts* t) {
   if (t->window < 0 || (t->window > 0 && t->window < d->tree_size)) return LS_ERR_INVALID_ARG;
   if (!(t->rope_theta >= 0.0) || !std::isfinite(t->rope_theta)) return LS_ERR_INVALID_ARG;
   if (t->rope_theta > 0.0 && t->rope_theta <= 1.0) return LS_ERR_INVALID_ARG;  // a base above 1
+  if (t->wait_limit_ns > kMaxWaitNs) return LS_ERR_INVALID_ARG;
   return LS_OK;
 }
 
@@ -99,6 +102,7 @@ int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_
   q.N = tree != nullptr && tree->cu_tree != nullptr ? tree->total_nodes : q.B * q.T;
   q.rope = with_tree && tree != nullptr && tree->rope_theta > 0.0 ? 1 : 0;
   q.window = with_tree && tree != nullptr ? tree->window : 0;
+  q.wait_ns = (int64_t)(tree != nullptr && tree->wait_limit_ns > 0 ? tree->wait_limit_ns : kDefaultWaitNs);
   if (q.g > ls::kUnitRows) return LS_ERR_UNSUPPORTED;
   q.tpu = ls::kUnitRows / q.g;
   q.rg = ls::ceil_div(q.T, q.tpu);
@@ -263,6 +267,7 @@ int run_partials(const void* q, const void* k_cache, const void* v_cache, const 
     ra.cu_tree = pa.cu_tree;
     ra.q_rot = reinterpret_cast<uint16_t*>(ws + lay.q_rot);
     ra.k_rot = reinterpret_cast<uint16_t*>(ws + lay.k_rot);
+    ra.rope_status = reinterpret_cast<uint32_t*>(ws + lay.rope_status);
     ra.log2_theta = std::log2(tree->rope_theta);
     ra.p = p;
     if (ls::launch_tree_rope(ra, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LS_ERR_CUDA;
@@ -270,6 +275,7 @@ int run_partials(const void* q, const void* k_cache, const void* v_cache, const 
     pa.k_tree = ra.k_rot;
     pa.after_prep = 1;
   }
+  pa.kv_rows = kv_rows;
   const cudaError_t e = ls::launch_partials(pa, kv_rows, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return LS_ERR_CUDA;
   return LS_OK;
@@ -310,6 +316,7 @@ int run_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verif
   ca.out = static_cast<uint16_t*>(out);
   ca.lse = lse;
   ca.status = reinterpret_cast<uint32_t*>(ws + lay.status);
+  ca.rope_status = p.rope ? reinterpret_cast<const uint32_t*>(ws + lay.rope_status) : nullptr;
   // the partials kernel ran just before unless a prefix-only call had no key at all
   ca.after_partials = with_tree || p.n_chunks > 0 ? 1 : 0;
   ca.p = p;
@@ -410,6 +417,7 @@ int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void
   if (all & ls::kErrLengths) return LS_ERR_LENGTHS;
   if (all & ls::kErrBadTree) return LS_ERR_BAD_TREE;
   if (all & ls::kErrTimeout) return LS_ERR_TIMEOUT;
+  if (all & ls::kErrIndex) return LS_ERR_INDEX;
   return LS_OK;
 }
 
@@ -423,6 +431,7 @@ const char* ls_status_string(int status) {
     case LS_ERR_BAD_TREE: return "tree_parent is not a rooted tree with parent[i] < i";
     case LS_ERR_TIMEOUT: return "a device-side wait timed out";
     case LS_ERR_LENGTHS: return "device cu_seqlens disagrees with the planned lengths";
+    case LS_ERR_INDEX: return "an index check of the index-checking build failed";
     default: return "unknown status";
   }
 }

@@ -64,6 +64,13 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
     rl = r;
     alt = unit_alternates(min(p.tpu, tree_n - u * p.tpu) * p.g);
     cbase = first + (kh * p.rg + u) * n;
+    // the row's chunks, its output row and (with RoPE) the tree kernel's word of its node
+    LS_DCHECK(err, b < p.B && kh < p.Hkv && u < p.rg && r < kUnitRows);
+    LS_DCHECK(err, !(writes && lengths_ok) || (cbase >= 0 && cbase + n <= p.n_chunks));
+    LS_DCHECK(err, !writes || (tree_base + i < p.N && out_row < (int64_t)p.N * p.Hq));
+#if defined(LS_DEBUG)
+    if (writes && a.rope_status != nullptr) err |= a.rope_status[(size_t)b * p.T + i];
+#endif
   }
   // the partials kernel may still be running: wait for its grid to finish
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -89,6 +96,8 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
         // every lane one partial's lse and status; up to kPrefetch outputs in flight
         float lx = -INFINITY;
         if (lane < nx) {
+          LS_DCHECK(err, cbase + ((x0 + lane) >> sh) < p.n_chunks &&
+                             part_row(x0 + lane) < (size_t)p.n_chunks * kUnitRows);
           lx = a.lse_part[part_row(x0 + lane)];
           err |= a.chunk_status[cbase + ((x0 + lane) >> sh)];
         }

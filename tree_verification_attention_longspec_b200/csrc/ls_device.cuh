@@ -29,6 +29,7 @@ struct PartialsArgs {
   float* lse_part;
   uint32_t* chunk_status;
   int32_t after_prep;  // q and k_tree are written by the tree kernel launched just before
+  int64_t kv_rows;     // rows of k_cache / v_cache (of the pages, for a paged cache)
   Plan p;
 };
 
@@ -42,6 +43,7 @@ struct TreeRopeArgs {
   const int32_t* cu_tree;
   uint16_t* q_rot;
   uint16_t* k_rot;
+  uint32_t* rope_status;  // index-checking builds: one word per CTA (node slot b * T + i)
   double log2_theta;  // log2 of the RoPE base
   Plan p;
 };
@@ -56,6 +58,7 @@ struct CombineArgs {
   uint16_t* out;
   float* lse;
   uint32_t* status;
+  const uint32_t* rope_status;  // index-checking builds, with RoPE: the tree kernel's words
   int32_t after_partials;  // launched right after the partials kernel: a programmatic dependent
   Plan p;
 };

@@ -34,6 +34,22 @@ constexpr int kPlanCu = 33;        // host lengths carried in the plan for batch
 constexpr uint32_t kErrBadTree = 1u;
 constexpr uint32_t kErrLengths = 2u;
 constexpr uint32_t kErrTimeout = 4u;
+constexpr uint32_t kErrIndex = 8u;  // index-checking (LS_DEBUG) builds: an address outside its extent
+
+// The index checks of the LS_DEBUG build: every TMA coordinate and global index the
+// kernels form is checked against the extent of the tensor it addresses, and a failed
+// check records kErrIndex in `flag` (reported through the call's status). Release
+// builds compile the checks away.
+#if defined(LS_DEBUG)
+#define LS_DCHECK(flag, ok)                    \
+  do {                                         \
+    if (!(ok)) (flag) |= ::ls::kErrIndex;      \
+  } while (0)
+#else
+#define LS_DCHECK(flag, ok) \
+  do {                      \
+  } while (0)
+#endif
 
 struct Plan {
   int32_t B, Hq, Hkv, d, T, g;  // T: tree nodes per sequence (the largest, with cu_tree)
@@ -56,6 +72,9 @@ struct Plan {
   // combine checks that the device array agrees. cu_n = 0: the device array is used.
   int32_t cu_n;
   int32_t cu_host[kPlanCu];
+  // Longest time any bounded device-side wait of the partials kernel may take before the
+  // call gives up and reports kErrTimeout (nanoseconds of %globaltimer).
+  int64_t wait_ns;
 };
 
 // The offsets the kernels address keys with: the plan's host copy, else the device array.
@@ -196,6 +215,7 @@ struct Layout {
   uint64_t chunk_status;  // u32   [n_chunks]
   uint64_t q_rot;         // bf16  [N][Hq][d]    rotated queries (rope only)
   uint64_t k_rot;         // bf16  [N][Hkv][d]   rotated tree keys (rope only)
+  uint64_t rope_status;   // u32   [B*T]         index-check result of each tree-kernel CTA (rope only)
   uint64_t total;
 };
 
@@ -217,6 +237,8 @@ LS_HD Layout make_layout(const Plan& p) {
   off = align256(off + nq);
   l.k_rot = off;
   off = align256(off + nk);
+  l.rope_status = off;
+  off = align256(off + (p.rope ? (uint64_t)p.B * p.T * 4 : 0));
   l.total = off;
   return l;
 }

@@ -27,7 +27,10 @@ constexpr int kMaxDevices = 64;
 // only a stand-in for the symbol, so its device address is looked up below.
 static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 
-void* g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device (set once)
+// Device address of g_scratch, per device, looked up once and kept for the life of the
+// process. cudaDeviceReset unloads this library's device code and a later call may find
+// the array elsewhere, so after a reset the process must not call this entry again.
+void* g_scratch_addr[kMaxDevices];
 
 }  // namespace
 

@@ -10,7 +10,7 @@
 // sequence's key list also takes the block of its T <= 128 tree keys, with every score
 // outside the row's ancestor-or-self set masked. A masked block is one more step of the
 // same online softmax, which is the log-sum-exp join itself. The CTA leaves its partial
-// (out normalised by its own sum, lse in the log2 domain) for the combine kernel.
+// (out normalised by its own sum; lse in the log2 domain) for the combine kernel.
 //
 // Ping-pong. Each query tile t has one softmax warpgroup, one score buffer S_t and one
 // output accumulator O_t in TMEM. The MMA thread walks the key blocks and, per block j,
@@ -39,8 +39,9 @@
 //   warp 9     MMA issuer (one thread): S = Q K^T (shared-memory operands, N = 128) and
 //              O += P V (P from TMEM, N = d), tcgen05.commit to mbarriers.
 // TMEM columns (512 allocated): S_t at 128 t, O_t at 256 + d t.
-// Every wait is bounded: on a timeout the CTA raises an abort flag, all roles drain
-// their in-flight copies and MMAs, TMEM is freed, and the chunk status reports it.
+// Every wait is bounded (the call's wait limit, 4 s by default): on a timeout the CTA
+// raises an abort flag, all roles drain their in-flight copies and MMAs, TMEM is freed,
+// and the chunk status reports it.
 #include <cudaTypedefs.h>
 
 #include "ls_device.cuh"
@@ -56,7 +57,9 @@ constexpr int kMmaWarp = 9;
 constexpr int kMaxSlots = 12;
 constexpr int kTiles = 2;  // 128-row query tiles per CTA
 constexpr int kHalf = 64;  // keys per P half
-constexpr uint64_t kTimeoutNs = 4000000000ull;
+// Draining after an abort waits for copies and MMAs that were issued and always
+// complete; its own bound is fixed (the call's wait limit may be far shorter).
+constexpr uint64_t kDrainNs = 4000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 static_assert(kUnitRows == kTiles * 128, "a unit is two 128-row tiles");
 
@@ -98,6 +101,7 @@ struct Bars {
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t tree_err;          // a parent link that is not a rooted tree's
+  uint32_t dbg;               // index-checking builds: kErrIndex once a check failed
   int16_t parent[kMaxTree];   // the sequence's tree (chunks that hold the tree block)
 };
 
@@ -128,11 +132,15 @@ __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t n, bool pred) {
 // Waits only on time (used to drain in-flight work after an abort).
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   uint32_t never = 0;
-  return mbar_wait_bounded(bar, parity, &never, kTimeoutNs);
+  return mbar_wait_bounded(bar, parity, &never, kDrainNs);
 }
 
-// P = 2^(s*cs - m) for 64 scores, packed to bf16 pairs; adds the values to (sum0, sum1).
-// EMU of every 4 pairs use the FMA-pipe exponential. Every block takes this one path,
+// P = 2^(s*cs - m) for 64 scores, packed to bf16 pairs; adds the values to (sum0, sum1)
+// and their bf16 roundings, the weights the PV product uses, to (rsum0, rsum1). The
+// output is normalised by the rounded sum, so that it is a convex combination of the
+// values with exactly those weights (their rounding, relative 2^-9 each, then cancels
+// where the values agree); the lse keeps the exact sum. EMU of every 4 pairs use the
+// FMA-pipe exponential. Every block takes this one path,
 // masked or not (one copy of the loop keeps the softmax's code small; a second, MUFU-only
 // copy for masked blocks cost 6% in time): a masked score (-inf) gives 0 on the MUFU
 // and 2^-125 on the FMA pipe, which clamps its input there, and 2^-125 is nothing next
@@ -140,7 +148,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 // and a later raise multiplies the sums by 2^-inf = 0).
 template <int EMU>
 __device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float m, uint32_t (&pk)[kHalf / 2],
-                                       float& sum0, float& sum1) {
+                                       float& sum0, float& sum1, float& rsum0, float& rsum1) {
   const float nm = -m;
 #pragma unroll
   for (int e = 0; e < kHalf / 2; ++e) {
@@ -154,6 +162,7 @@ __device__ __forceinline__ void make_p(const float (&s)[kHalf], float cs, float 
     }
     add2(sum0, sum1, p0, p1);
     pk[e] = pack_bf16x2(p0, p1);
+    add_bf16x2_to_f32(rsum0, rsum1, pk[e]);
   }
 }
 
@@ -211,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   const PartialsArgs& a = P.a;
   const Plan& p = a.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint64_t wait_ns = (uint64_t)p.wait_ns;  // limit of every bounded wait below
 
   const int32_t* cu = plan_cu(p, a.cu);  // kernel parameters when the host gave lengths
   const ChunkCoord c = locate_chunk(p, cu, blockIdx.x);
@@ -248,166 +258,198 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     return;
   }
 
-  if (tid == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < C::kSlots; ++s) {
-      mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->empty[s], 1);
+  volatile uint32_t* abort = &bars->abort;
+  // ------------------------------------------------------------------ TMA producer state
+  // Ring order = consumption order: K(0), V(0), K(1), V(1), ... The whole warp walks the
+  // blocks; lane 0 arms the barriers and issues whole-block boxes, and for a paged cache
+  // the lanes issue the block's page boxes (and read their page-table entries) at once.
+  // The producer sets up the barriers and issues Q and K(0) before the CTA-wide barrier,
+  // so that the first tiles are in flight while the other warps set up.
+  // Q: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows past the
+  // batch's last node read as zeros)
+  auto load_q = [&]() {
+#if defined(LS_DEBUG)
+    // the unit's existing nodes lie inside q (the box rows after them read zeros)
+    if (lane == 0 && !(tok0 >= 0 && tok0 < tree_n && tree_base >= 0 && tree_base + tree_n <= p.N)) bars->dbg = kErrIndex;
+#endif
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn)
+        tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
+                    tree_base + tok0);
     }
-    for (int t = 0; t < kTiles; ++t) {
-      mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t][0], 128);
-      mbar_init(&bars->p_full[t][1], 128);
+  };
+  // When the tree kernel writes q and k_tree (rotated), this grid may start before
+  // that grid ends: the prefix loads go ahead, Q and the tree block wait for it.
+  bool prior_done = !a.after_prep;
+  auto wait_prior = [&]() {
+    if (!prior_done) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      prior_done = true;
     }
-    mbar_init(&bars->o_full[0], 1);
-    mbar_init(&bars->o_full[1], 1);
-    bars->abort = 0u;
-    bars->tree_err = 0u;
-    fence_mbar_init();
+  };
+  bool q_loaded = false;
+  // a page box is bh rows (the page, or 128 rows of a larger page); lane l issues box
+  // l / kPanels, panel l % kPanels
+  const int bh = paged ? (a.page_size < kBlockN ? a.page_size : kBlockN) : kBlockN;
+  const int n_boxes = (kBlockN / bh) * C::kPanels;
+  const int n_pages = paged ? (seq_len + a.page_size - 1) / a.page_size : 0;
+  int issued = 0, slot = 0, use = 0;
+  // the MMA thread's order: K(j), V(j) for j = 0, 1, ...; with alternate blocks K(0),
+  // K(1), then V(j) and K(j + 2) for j = 0, 1, ... (no K past the last block)
+  const int n_loads = 2 * nbt;
+  const int pro = nbt < 2 ? nbt : 2, pairs = nbt > 2 ? nbt - 2 : 0;
+  // Issues load `ld` of the ring once its slot is free; false if the wait gave up.
+  auto issue_load = [&](int ld) -> bool {
+    int j, kv;
+    if (!alt) {
+      j = ld >> 1;
+      kv = ld & 1;
+    } else if (ld < pro) {
+      j = ld;
+      kv = 0;
+    } else if (ld - pro < 2 * pairs) {
+      const int r = ld - pro;
+      j = (r >> 1) + ((r & 1) ? 2 : 0);
+      kv = (r & 1) ? 0 : 1;
+    } else {
+      j = pairs + (ld - pro - 2 * pairs);
+      kv = 1;
+    }
+    // prefix block j, or the tree block: the sequence's nodes (the rows after them
+    // belong to the next sequence or lie past the tensor, read as zeros; masked)
+    const bool tree = j == nb;
+    int row = c.seq_offset + c.key_begin + j * kBlockN;
+    if (j == nb - 1) row -= tail_shift;  // the box ends at the sequence end
+    if (tree) {
+      row = tree_base;
+      wait_prior();
+    }
+    const bool pieces = paged && !tree;  // the block's rows come page by page
+    // this lane's page box of the block: a page-table entry is only a TMA coordinate,
+    // so a bad one reads zeros or another page, never outside the cache; boxes past
+    // the sequence end read its last page (masked)
+    int prow = 0;
+    const int pc = lane / C::kPanels, pn_l = lane % C::kPanels;
+    if (pieces && lane < n_boxes) {
+      const int key = c.key_skip + c.key_begin + j * kBlockN + pc * bh;
+      int lp = key / a.page_size;
+      if (lp >= n_pages) lp = n_pages - 1;
+      if (lp >= a.max_pages) lp = a.max_pages - 1;
+      prow = a.page_table[(size_t)c.b * a.max_pages + lp] * a.page_size + key % a.page_size;
+    }
+#if defined(LS_DEBUG)
+    {
+      // the rows of the block that are not masked must lie inside the sequence (inside the
+      // tree for the tree block) and every box inside the tensor's data
+      uint32_t bad = 0u;
+      if (tree) {
+        LS_DCHECK(bad, tree_base >= 0 && tree_base + tree_n <= p.N);
+      } else if (!pieces) {
+        const int lo = j == nb - 1 ? tail_shift : 0;
+        LS_DCHECK(bad, j >= 0 && j < nb);
+        LS_DCHECK(bad, row + lo >= c.seq_offset && row + kBlockN <= cu[c.b + 1]);
+        LS_DCHECK(bad, row + kBlockN <= cu[p.B] && (int64_t)row + kBlockN <= a.kv_rows);
+      } else if (lane < n_boxes) {
+        const int key = c.key_skip + c.key_begin + j * kBlockN + pc * bh;
+        if (key < c.key_skip + c.key_end) {  // a box with keys of the sequence (else masked)
+          const int lp = key / a.page_size;
+          LS_DCHECK(bad, lp < n_pages && lp < a.max_pages && c.b < p.B);
+          const int32_t pe = a.page_table[(size_t)c.b * a.max_pages + lp];
+          LS_DCHECK(bad, pe >= 0 && (int64_t)pe * a.page_size + bh <= a.kv_rows);
+        }
+      }
+      bad = __reduce_or_sync(0xffffffffu, bad);
+      if (lane == 0 && bad) bars->dbg = kErrIndex;
+    }
+#endif
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, wait_ns)))
+      return false;
+    if (lane == 0) mbar_arrive_expect_tx(&bars->full[slot], C::kTileBytes);
+    __syncwarp();
+    uint8_t* dst = smem + C::kSlotOff + slot * C::kTileBytes;
+    const CUtensorMap* map = tree ? (kv ? &P.tmap_vt : &P.tmap_kt) : (kv ? &P.tmap_v : &P.tmap_k);
+    if (!pieces) {
+      if (lane == 0) {
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
+      }
+    } else if (lane < n_boxes) {
+      tma_load_3d(dst + pn_l * C::kPanelBytes + pc * bh * 128, map, &bars->full[slot], pn_l * 64, c.kh, prow);
+    }
+    ++issued;
+    if (++slot == C::kSlots) {
+      slot = 0;
+      ++use;
+    }
+    return true;
+  };
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      mbar_init(&bars->q_full, 1);
+      for (int s = 0; s < C::kSlots; ++s) {
+        mbar_init(&bars->full[s], 1);
+        mbar_init(&bars->empty[s], 1);
+      }
+      for (int t = 0; t < kTiles; ++t) {
+        mbar_init(&bars->s_full[t], 1);
+        mbar_init(&bars->p_full[t][0], 128);
+        mbar_init(&bars->p_full[t][1], 128);
+      }
+      mbar_init(&bars->o_full[0], 1);
+      mbar_init(&bars->o_full[1], 1);
+      bars->abort = 0u;
+      bars->tree_err = 0u;
+      bars->dbg = 0u;
+      fence_mbar_init();
+      tma_prefetch_map(&P.tmap_q);
+      tma_prefetch_map(&P.tmap_k);
+      tma_prefetch_map(&P.tmap_v);
+      tma_prefetch_map(&P.tmap_o);
+      if (has_tree) {
+        tma_prefetch_map(&P.tmap_kt);
+        tma_prefetch_map(&P.tmap_vt);
+      }
+    }
+    __syncwarp();
+    // K(0) first, then Q (unless Q waits for the tree kernel): at start-up every CTA asks
+    // for just these two, so they arrive quickly instead of sharing the memory system with
+    // the whole ring's fill. A fresh barrier never makes the first wait give up.
+    issue_load(0);
+    if (prior_done) {
+      load_q();
+      q_loaded = true;
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
-    tma_prefetch_map(&P.tmap_q);
-    tma_prefetch_map(&P.tmap_k);
-    tma_prefetch_map(&P.tmap_v);
-    tma_prefetch_map(&P.tmap_o);
-    if (has_tree) {
-      tma_prefetch_map(&P.tmap_kt);
-      tma_prefetch_map(&P.tmap_vt);
-    }
-  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tbase = bars->tmem_base;
-  volatile uint32_t* abort = &bars->abort;
   // the tree/combine kernel may start its own prologue now; it waits for this grid's
   // results before it reads them
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == kProducerWarp) {
-    // ------------------------------------------------------------------ TMA producer
-    // Ring order = consumption order: K(0), V(0), K(1), V(1), ... The whole warp walks the
-    // blocks; lane 0 arms the barriers and issues whole-block boxes, and for a paged cache
-    // the lanes issue the block's page boxes (and read their page-table entries) at once.
     {
-      // Q: one box per 64-column panel, tpu nodes x g heads of kv head kh (rows past the
-      // batch's last node read as zeros)
-      auto load_q = [&]() {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&bars->q_full, C::kPanels * 128 * p.g * p.tpu);
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_4d(smem + C::kQOff + pn * C::kQPanelBytes, &P.tmap_q, &bars->q_full, pn * 64, 0, c.kh,
-                        tree_base + tok0);
-        }
-      };
-      // When the tree kernel writes q and k_tree (rotated), this grid may start before
-      // that grid ends: the prefix loads go ahead, Q and the tree block wait for it.
-      bool prior_done = !a.after_prep;
-      auto wait_prior = [&]() {
-        if (!prior_done) {
-          asm volatile("griddepcontrol.wait;" ::: "memory");
-          prior_done = true;
-        }
-      };
-      bool q_loaded = false;
-      if (prior_done) {
+      bool ok = true;
+      if (!q_loaded) {
+        wait_prior();
         load_q();
         q_loaded = true;
       }
-      // a page box is bh rows (the page, or 128 rows of a larger page); lane l issues box
-      // l / kPanels, panel l % kPanels
-      const int bh = paged ? (a.page_size < kBlockN ? a.page_size : kBlockN) : kBlockN;
-      const int n_boxes = (kBlockN / bh) * C::kPanels;
-      const int n_pages = paged ? (seq_len + a.page_size - 1) / a.page_size : 0;
-      int issued = 0, slot = 0, use = 0;
-      bool ok = true;
-      // the MMA thread's order: K(j), V(j) for j = 0, 1, ...; with alternate blocks K(0),
-      // K(1), then V(j) and K(j + 2) for j = 0, 1, ... (no K past the last block)
-      const int n_loads = 2 * nbt;
-      const int pro = nbt < 2 ? nbt : 2, pairs = nbt > 2 ? nbt - 2 : 0;
-      for (int ld = 0; ld < n_loads && ok; ++ld) {
-        int j, kv;
-        if (!alt) {
-          j = ld >> 1;
-          kv = ld & 1;
-        } else if (ld < pro) {
-          j = ld;
-          kv = 0;
-        } else if (ld - pro < 2 * pairs) {
-          const int r = ld - pro;
-          j = (r >> 1) + ((r & 1) ? 2 : 0);
-          kv = (r & 1) ? 0 : 1;
-        } else {
-          j = pairs + (ld - pro - 2 * pairs);
-          kv = 1;
-        }
-        // prefix block j, or the tree block: the sequence's nodes (the rows after them
-        // belong to the next sequence or lie past the tensor, read as zeros; masked)
-        const bool tree = j == nb;
-        int row = c.seq_offset + c.key_begin + j * kBlockN;
-        if (j == nb - 1) row -= tail_shift;  // the box ends at the sequence end
-        if (tree) {
-          row = tree_base;
-          wait_prior();
-        }
-        const bool pieces = paged && !tree;  // the block's rows come page by page
-        // this lane's page box of the block: a page-table entry is only a TMA coordinate,
-        // so a bad one reads zeros or another page, never outside the cache; boxes past
-        // the sequence end read its last page (masked)
-        int prow = 0;
-        const int pc = lane / C::kPanels, pn_l = lane % C::kPanels;
-        if (pieces && lane < n_boxes) {
-          const int key = c.key_skip + c.key_begin + j * kBlockN + pc * bh;
-          int lp = key / a.page_size;
-          if (lp >= n_pages) lp = n_pages - 1;
-          if (lp >= a.max_pages) lp = a.max_pages - 1;
-          prow = a.page_table[(size_t)c.b * a.max_pages + lp] * a.page_size + key % a.page_size;
-        }
-        {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->empty[slot], (use & 1) ^ 1, abort, kTimeoutNs))) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) mbar_arrive_expect_tx(&bars->full[slot], C::kTileBytes);
-          __syncwarp();
-          uint8_t* dst = smem + C::kSlotOff + slot * C::kTileBytes;
-          const CUtensorMap* map = tree ? (kv ? &P.tmap_vt : &P.tmap_kt) : (kv ? &P.tmap_v : &P.tmap_k);
-          if (!pieces) {
-            if (lane == 0) {
-#pragma unroll
-              for (int pn = 0; pn < C::kPanels; ++pn)
-                tma_load_3d(dst + pn * C::kPanelBytes, map, &bars->full[slot], pn * 64, c.kh, row);
-            }
-          } else if (lane < n_boxes) {
-            tma_load_3d(dst + pn_l * C::kPanelBytes + pc * bh * 128, map, &bars->full[slot], pn_l * 64, c.kh, prow);
-          }
-          ++issued;
-          if (++slot == C::kSlots) {
-            slot = 0;
-            ++use;
-          }
-          // K(0) alone first: at start-up every CTA asks for just Q and one tile, so those
-          // arrive quickly instead of sharing the memory system with the whole ring's fill
-          if (issued == 1 && !q_loaded) {
-            wait_prior();
-            load_q();
-            q_loaded = true;
-          }
-          if (issued == 1 && !__all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[0], 0, abort, kTimeoutNs))) {
-            ok = false;
-            break;
-          }
-        }
-      }
-      // make sure no copy is still writing shared memory when the CTA ends (Q was
-      // issued unless the loop stopped before its first load)
+      // the rest of the ring once K(0) has landed
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars->full[0], 0, abort, wait_ns))) ok = false;
+      for (int ld = 1; ld < n_loads && ok; ++ld) ok = issue_load(ld);
+      // make sure no copy is still writing shared memory when the CTA ends
       if (lane == 0) {
-        if (q_loaded) drain_wait(&bars->q_full, 0);
+        drain_wait(&bars->q_full, 0);
         const int first = issued > C::kSlots ? issued - C::kSlots : 0;
         for (int seq = first; seq < issued; ++seq)
           drain_wait(&bars->full[seq % C::kSlots], (seq / C::kSlots) & 1);
@@ -431,6 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       // as a value that fails the walk's checks
       if (has_tree || win_rows) {
         for (int x = tid; x < tree_n; x += 256) {
+#if defined(LS_DEBUG)
+          if (!(tree_base + x < p.N)) bars->dbg = kErrIndex;
+#endif
           const int32_t pp = a.parent[(size_t)tree_base + x];
           bars->parent[x] = (int16_t)(pp >= -1 && pp < tree_n ? pp : kMaxTree);
         }
@@ -478,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           }
         };
         auto wait = [&](uint64_t* bar, uint32_t parity) {
-          const bool got = mbar_wait_bounded(bar, parity, abort, kTimeoutNs);
+          const bool got = mbar_wait_bounded(bar, parity, abort, wait_ns);
           if (got) tc_fence_after_sync();
           return got;
         };
@@ -576,7 +621,9 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const uint32_t tS = tbase + lane_base + C::kColS + t * kBlockN;
       const uint32_t tO = tbase + lane_base + C::kColO + t * D;
       const float cs = p.scale_log2;
-      float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of this row
+      // running max (log2 units) of this row, its sum of weights and the sum of their
+      // bf16 roundings (the weights in O_t)
+      float m = -INFINITY, l = 0.f, lr = 0.f;
       const int ur = alt ? row : t * 128 + row;  // row of the unit (both tiles' rows when alternating)
       const bool has_row = ur < rows_here;
       const int node = tok0 + ur / p.g;   // its tree node
@@ -596,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
       const int n_mine = alt ? (nbt - t + 1) / 2 : nbt;
       for (int i = 0; i < n_mine; ++i) {
         const int j = alt ? 2 * i + t : i;  // the block
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], i & 1, abort, kTimeoutNs));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[t], i & 1, abort, wait_ns));
         if (!ok) break;
         tc_fence_after_sync();
         int shift = j == nb - 1 ? tail_shift : 0;          // masked leading columns (this row)
@@ -646,10 +693,10 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         // a row that has seen no visible key yet (a padding row of a tree-only chunk)
         // keeps m = -inf; its P is 0 against any finite reference
         const float m_ref = m_new == -INFINITY ? 0.f : m_new;
-        float sum0 = 0.f, sum1 = 0.f;
+        float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
         {
           uint32_t pk[kHalf / 2];
-          make_p<EMU>(lo, cs, m_ref, pk, sum0, sum1);
+          make_p<EMU>(lo, cs, m_ref, pk, sum0, sum1, rsum0, rsum1);
           if (any_raise) {
             // the maximum moved up: rescale what O_t and l hold. O_t is idle: every PV of
             // this tile issued before S_t(j) has completed (s_full), and PV_t(j) waits for
@@ -667,6 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
               }
             }
             l *= f;
+            lr *= f;
             m = m_new;
           }
           tmem_st32(tS, pk);  // P over keys 0..63 -> columns 0..31
@@ -690,16 +738,17 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         }
         {
           uint32_t pk[kHalf / 2];
-          make_p<EMU>(hi, cs, m_ref, pk, sum0, sum1);
+          make_p<EMU>(hi, cs, m_ref, pk, sum0, sum1, rsum0, rsum1);
           tmem_st32(tS + 32, pk);  // keys 64..127 -> columns 32..63
           tmem_wait_st();
           tc_fence_before_sync();
           mbar_arrive(&bars->p_full[t][1]);
         }
         l += sum0 + sum1;
+        lr += rsum0 + rsum1;
       }
       // -------------------------------------------------------------- epilogue
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full[t], 0, abort, kTimeoutNs));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->o_full[t], 0, abort, wait_ns));
       // Each warpgroup stages its normalised 128 x D tile in shared memory as D/32 panels
       // of 128 rows x 128 B, swizzled like the tensor map (16-byte chunk q of row r at
       // q ^ (r & 7): conflict-free for the per-row writes), and one thread stores the
@@ -712,7 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         tc_fence_after_sync();
         constexpr int kOPanels = D / 32;  // 128-byte panels of an fp32 row
         uint8_t* stage = smem + (t == 0 ? C::kQOff : C::kSlotOff);
-        const float inv = 1.f / l;
+        const float inv = 1.f / lr;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {  // panel q = columns [32 q, 32 q + 32)
           uint32_t r[32];
@@ -725,6 +774,10 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
                             __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
         // this tile's partial: rows [128 t, 128 t + 128) of the chunk's slot
+#if defined(LS_DEBUG)
+        // the partial's rows stay inside the chunk's slot of o_part / lse_part
+        if (!((int64_t)blockIdx.x < p.n_chunks && t * 128 + row < kUnitRows)) bars->dbg = kErrIndex;
+#endif
         if (has_row) a.lse_part[(size_t)blockIdx.x * kUnitRows + t * 128 + row] = m + log2f(l);
         fence_proxy_async_smem();  // the staged tile is read by the TMA unit
         asm volatile("bar.sync %0, 128;" ::"r"(2 + t) : "memory");
@@ -745,7 +798,8 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
     tc_fence_after_sync();
     tmem_dealloc(tbase, C::kTmemCols);
   }
-  if (tid == 0) a.chunk_status[blockIdx.x] = (bars->abort ? kErrTimeout : 0u) | (bars->tree_err ? kErrBadTree : 0u);
+  if (tid == 0)
+    a.chunk_status[blockIdx.x] = (bars->abort ? kErrTimeout : 0u) | (bars->tree_err ? kErrBadTree : 0u) | bars->dbg;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

@@ -50,31 +50,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Tests four barrier phases at once (the four probes are independent, so they are in
-// flight together); true if all four have completed.
-__device__ __forceinline__ bool mbar_try_wait4(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
-                                               uint32_t p2, uint64_t* b3, uint32_t p3) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred q0, q1, q2, q3;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q0, [%1], %2;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q1, [%3], %4;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q2, [%5], %6;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 q3, [%7], %8;\n\t"
-      "and.pred q0, q0, q1;\n\t"
-      "and.pred q2, q2, q3;\n\t"
-      "and.pred q0, q0, q2;\n\t"
-      "selp.u32 %0, 1, 0, q0;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1), "r"(smem_u32(b2)), "r"(p2), "r"(smem_u32(b3)),
-        "r"(p3)
-      : "memory");
-  return ok != 0;
-}
-
 // Waits for the phase of `bar` with the given parity to complete. Gives up after
 // `timeout_ns` of global time, or as soon as another thread has raised *abort, and
-// then returns false (raising *abort itself on a timeout). Never spins forever.
+// then returns false (raising *abort itself on a timeout). Never spins forever: each
+// probe that the barrier does not complete returns after a time limit of the hardware's,
+// and the loop checks the clock between probes.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile uint32_t* abort, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -93,15 +73,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-
-// 16-byte global -> shared copy that bypasses registers (LDGSTS); src_bytes = 0 writes
-// zeros and reads nothing. Completes at cp_async_wait_all().
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
@@ -259,24 +230,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
-      "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
-      "%56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
-        "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
-        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
-        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
-        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr));
-}
-
 // ----------------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -345,6 +298,16 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, floa
         "f"(6.932609677e-01f), "f"(2.426111251e-01f), "f"(5.517166853e-02f));
   p0 = __uint_as_float(q0 + (t0 << 23));
   p1 = __uint_as_float(q1 + (t1 << 23));
+}
+
+// (s0, s1) += the two bf16 halves of `packed` (low half into s0), in fp32.
+__device__ __forceinline__ void add_bf16x2_to_f32(float& s0, float& s1, uint32_t packed) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\t"
+      "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "r"(packed));
 }
 
 // (lo, hi) -> packed bf16x2 with `lo` in the low half, round to nearest even.

@@ -61,7 +61,12 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
   const int b = blockIdx.x / p.T, i = blockIdx.x % p.T;
   int base = 0, n = 0;
   tree_range(p, a.cu_tree, b, &base, &n);
-  if (i >= n) return;
+  if (i >= n) {  // a node slot past the sequence's tree
+#if defined(LS_DEBUG)
+    if (threadIdx.x == 0) a.rope_status[blockIdx.x] = 0u;
+#endif
+    return;
+  }
   const int tid = threadIdx.x;
   const int half = p.d / 2;
   const int groups = half / 8;  // items: (head, group of 8 pairs); q heads first, then k_tree's
@@ -75,11 +80,14 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
     const int hh = it / groups, e0 = (it % groups) * 8;
     return hh < p.Hq ? a.q_rot + (node * p.Hq + hh) * p.d + e0 : a.k_rot + (node * p.Hkv + (hh - p.Hq)) * p.d + e0;
   };
+  uint32_t bad = 0u;  // index-checking builds: this CTA's failed checks
+  LS_DCHECK(bad, b < p.B && node < (size_t)p.N);
   uint4 lo[kPrefetch], hi[kPrefetch];
 #pragma unroll
   for (int k = 0; k < kPrefetch; ++k) {
     const int it = tid + k * kRopeThreads;
     if (it < items) {
+      LS_DCHECK(bad, it / groups < p.Hq + p.Hkv && (it % groups) * 8 + 8 <= half);
       lo[k] = *reinterpret_cast<const uint4*>(src_of(it));
       hi[k] = *reinterpret_cast<const uint4*>(src_of(it) + half);
     }
@@ -88,6 +96,7 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
   __shared__ int32_t anc[2][kMaxTree], dist[2][kMaxTree];
   __shared__ float cos_s[64], sin_s[64];
   if (tid < n) {
+    LS_DCHECK(bad, base + tid < p.N);
     const int32_t pp = a.parent[(size_t)base + tid];
     const bool link = tid > 0 && pp >= 0 && pp < tid;  // a valid link one level up
     anc[0][tid] = link ? pp : tid;                     // the root (or a bad link) points at itself
@@ -133,6 +142,7 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
     }
   }
   for (int it = tid + kPrefetch * kRopeThreads; it < items; it += kRopeThreads) {  // large head counts
+    LS_DCHECK(bad, it / groups < p.Hq + p.Hkv);
     const uint4 l1 = *reinterpret_cast<const uint4*>(src_of(it));
     const uint4 h1 = *reinterpret_cast<const uint4*>(src_of(it) + half);
     uint4 olo, ohi;
@@ -140,6 +150,11 @@ __global__ void __launch_bounds__(kRopeThreads) tree_rope_kernel(TreeRopeArgs a)
     *reinterpret_cast<uint4*>(dst_of(it)) = olo;
     *reinterpret_cast<uint4*>(dst_of(it) + half) = ohi;
   }
+#if defined(LS_DEBUG)
+  // one word per node slot, read by the combine for the rows of this node
+  bad = __syncthreads_or(bad) ? kErrIndex : 0u;
+  if (tid == 0) a.rope_status[blockIdx.x] = bad;
+#endif
 }
 
 }  // namespace
