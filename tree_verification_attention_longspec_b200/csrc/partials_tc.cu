@@ -522,11 +522,16 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             umma_ts(tO, tP + kk * 8, dv + kk * (2048 / 16), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
         };
+        // P written by the softmax warps' tcgen05.st: their wait::st, fence and arrive pair
+        // with this wait and the fence after it before an MMA reads P
         auto wait = [&](uint64_t* bar, uint32_t parity) {
           const bool got = mbar_wait_bounded(bar, parity, abort, wait_ns);
           if (got) tc_fence_after_sync();
           return got;
         };
+        // Q, K, V written by TMA: the barrier's transaction count completes once the bytes
+        // are in shared memory, where the MMAs read them; no tcgen05 fence is needed
+        auto wait_tma = [&](uint64_t* bar, uint32_t parity) { return mbar_wait_bounded(bar, parity, abort, wait_ns); };
         int slot = 0, use = 0;  // ring position of the next tile, in consumption order
         auto advance = [&]() {
           if (++slot == C::kSlots) {
@@ -534,12 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             use ^= 1;
           }
         };
-        bool ok = wait(&bars->q_full, 0);
+        bool ok = wait_tma(&bars->q_full, 0);
         if (alt) {
           // alternate blocks: tile t takes blocks t, t + 2, ...; S_t = Q K(t)^T first, then
           // for j = 0, 1, ...: PV of block j for tile j % 2 and that tile's next QK^T
           for (int t = 0; t < kTiles && t < nbt && ok; ++t) {
-            ok = wait(&bars->full[slot], use);
+            ok = wait_tma(&bars->full[slot], use);
             if (!ok) break;
             issue_qk(t, slot);
             umma_commit(&bars->empty[slot]);
@@ -547,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           }
           for (int j = 0; j < nbt && ok; ++j) {
             const int t = j & 1, i = j >> 1;  // tile and its own block count
-            ok = wait(&bars->full[slot], use);  // V(j)
+            ok = wait_tma(&bars->full[slot], use);  // V(j)
             if (!ok) break;
             const int sv = slot;
             advance();
@@ -559,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             issue_pv(t, sv, i, 1);
             umma_commit(&bars->empty[sv]);
             if (j + 2 < nbt) {
-              ok = wait(&bars->full[slot], use);  // K(j + 2)
+              ok = wait_tma(&bars->full[slot], use);  // K(j + 2)
               if (!ok) break;
               issue_qk(t, slot);
               umma_commit(&bars->empty[slot]);
@@ -570,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           }
         }
         if (ok && !alt) {
-          ok = wait(&bars->full[slot], use);  // K(0)
+          ok = wait_tma(&bars->full[slot], use);  // K(0)
           if (ok) {
             issue_qk(0, slot);
             issue_qk(1, slot);
@@ -584,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
           const bool more = j + 1 < nbt;
           const int sk = slot, uk = use;  // K(j+1), when there is one
           const uint32_t pp = j & 1;
-          ok = wait(&bars->full[sv], uv);
+          ok = wait_tma(&bars->full[sv], uv);
           for (int t = 0; t < kTiles && ok; ++t) {
             ok = wait(&bars->p_full[t][0], pp);
             if (!ok) break;
@@ -597,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             if (t == 1) umma_commit(&bars->empty[sv]);
             if (!more && t == 0) umma_commit(&bars->o_full[0]);  // tile 0's epilogue may start
             if (more) {
-              if (t == 0) ok = wait(&bars->full[sk], uk);
+              if (t == 0) ok = wait_tma(&bars->full[sk], uk);
               if (!ok) break;
               issue_qk(t, sk);
             }
