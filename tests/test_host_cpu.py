@@ -52,11 +52,20 @@ def test_prefix_only_plan_covers_every_prefix_block_once(plan_check, B, Hq, Hkv,
     assert r.returncode == 0, r.stdout + r.stderr
 
 
-def test_plan_check_catches_an_uncovered_tree_block(plan_check):
+def test_plan_check_catches_a_plan_too_short_for_the_keys(plan_check):
     # uniform plan of 3 chunks of 5 blocks: 1920 keys need 15 prefix blocks and the tree
-    # block, 16 in all, so the tree block of that sequence is left out
+    # block, 16 in all; spread evenly over 3 chunks one of them needs 6 blocks, more than
+    # the plan's C (on the device the combine reports such lengths as LS_ERR_LENGTHS)
     r = subprocess.run([plan_check, "1", "4", "1", "16", "5", "3", "1920"], capture_output=True, text=True)
-    assert r.returncode == 1 and "covered 0 times" in r.stdout
+    assert r.returncode == 1 and "too long" in r.stdout
+
+
+def test_plan_check_catches_a_missing_block(plan_check):
+    # a prefix-only plan of one chunk of 5 blocks over 6 blocks of keys: the sixth block is
+    # covered by no chunk (the even split of 6 blocks over 1 chunk is 6 > C first)
+    env = dict(os.environ, PLAN_CHECK_NO_TREE="1")
+    r = subprocess.run([plan_check, "1", "4", "1", "16", "5", "1", "700"], capture_output=True, text=True, env=env)
+    assert r.returncode == 1 and ("too long" in r.stdout or "covered 0 times" in r.stdout)
 
 
 def test_random_plans(plan_check):

@@ -80,7 +80,10 @@ int check_tree(const ls_verify_dims* d, const ls_tree_opts* t) {
 // Chooses the chunk length C (in 128-key blocks) that minimises the estimated time of
 // the partials kernel: waves of `slots` CTAs, each wave as long as its longest chunk
 // plus a fixed per-chunk cost for loading Q and writing the partial. A sequence's key
-// list is its prefix blocks plus one tree block.
+// list is its prefix blocks plus one tree block, cut into ceil(blocks / C) chunks of
+// nearly equal length (none longer than C). The estimate is closed-form: the plan is
+// made on every call, so it must cost microseconds, not the milliseconds that simulating
+// the grid's schedule would.
 int make_plan(const ls_verify_dims* d, Plan* p, bool with_tree = true, const ls_tree_opts* tree = nullptr) {
   int rc = check_dims(d);
   if (rc != LS_OK) return rc;
@@ -196,10 +199,15 @@ namespace {
 int run_partials(const void* q, const void* k_cache, const void* v_cache, const void* k_tree, const void* v_tree,
                  const int32_t* tree_parent, const int32_t* cu_seqlens, const ls_verify_dims* dims,
                  const ls_paged_kv* pg, void* workspace, size_t workspace_bytes, void* stream,
-                 bool with_tree = true, const ls_tree_opts* tree = nullptr) {
+                 bool with_tree = true, const ls_tree_opts* tree = nullptr, const Plan* planned = nullptr) {
+  // the caller's plan for these arguments when it made one already (one plan per call)
   Plan p;
-  int rc = make_plan(dims, &p, with_tree, tree);
-  if (rc != LS_OK) return rc;
+  if (planned != nullptr) {
+    p = *planned;
+  } else {
+    const int rc0 = make_plan(dims, &p, with_tree, tree);
+    if (rc0 != LS_OK) return rc0;
+  }
   if (q == nullptr || !aligned16(q) || cu_seqlens == nullptr || !aligned4(cu_seqlens)) return LS_ERR_INVALID_ARG;
   if (with_tree) {
     if (k_tree == nullptr || v_tree == nullptr || !aligned16(k_tree) || !aligned16(v_tree))
@@ -297,10 +305,15 @@ int ls_verify_attn_partials(const void* q, const void* k_cache, const void* v_ca
 namespace {
 
 int run_combine(const int32_t* cu_seqlens, void* out, float* lse, const ls_verify_dims* dims, void* workspace,
-                size_t workspace_bytes, void* stream, bool with_tree, const ls_tree_opts* tree = nullptr) {
+                size_t workspace_bytes, void* stream, bool with_tree, const ls_tree_opts* tree = nullptr,
+                const Plan* planned = nullptr) {
   Plan p;
-  int rc = make_plan(dims, &p, with_tree, tree);
-  if (rc != LS_OK) return rc;
+  if (planned != nullptr) {
+    p = *planned;
+  } else {
+    const int rc0 = make_plan(dims, &p, with_tree, tree);
+    if (rc0 != LS_OK) return rc0;
+  }
   if (out == nullptr || !aligned16(out)) return LS_ERR_INVALID_ARG;
   if (cu_seqlens == nullptr || lse == nullptr || !aligned4(cu_seqlens) || !aligned4(lse)) return LS_ERR_INVALID_ARG;
   const ls::Layout lay = ls::make_layout(p);
@@ -346,9 +359,9 @@ int ls_cross_attn(const void* q, const void* k_cache, const void* v_cache, const
   if (rc != LS_OK) return rc;
   if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
   rc = run_partials(q, k_cache, v_cache, nullptr, nullptr, nullptr, cu_seqlens, dims, nullptr, workspace,
-                    workspace_bytes, stream, false);
+                    workspace_bytes, stream, false, nullptr, &p);
   if (rc != LS_OK) return rc;
-  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, false);
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, false, nullptr, &p);
 }
 
 int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache, const void* k_tree,
@@ -360,10 +373,10 @@ int ls_verify_attn(const void* q, const void* k_cache, const void* v_cache, cons
   int rc = make_plan(dims, &p);
   if (rc != LS_OK) return rc;
   if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
-  rc = ls_verify_attn_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, workspace,
-                               workspace_bytes, stream);
+  rc = run_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, nullptr, workspace,
+                    workspace_bytes, stream, true, nullptr, &p);
   if (rc != LS_OK) return rc;
-  return ls_verify_attn_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream);
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, true, nullptr, &p);
 }
 
 int ls_verify_attn_paged(const void* q, const void* k_pages, const void* v_pages, const ls_paged_kv* paged,
@@ -376,9 +389,9 @@ int ls_verify_attn_paged(const void* q, const void* k_pages, const void* v_pages
   if (paged == nullptr) return LS_ERR_INVALID_ARG;
   if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
   rc = run_partials(q, k_pages, v_pages, k_tree, v_tree, tree_parent, cu_seqlens, dims, paged, workspace,
-                    workspace_bytes, stream);
+                    workspace_bytes, stream, true, nullptr, &p);
   if (rc != LS_OK) return rc;
-  return ls_verify_attn_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream);
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, true, nullptr, &p);
 }
 
 size_t ls_verify_attn_ex_workspace_size(const ls_verify_dims* dims, const ls_tree_opts* tree) {
@@ -396,9 +409,9 @@ int ls_verify_attn_ex(const void* q, const void* k_cache, const void* v_cache, c
   if (rc != LS_OK) return rc;
   if (out == nullptr || !aligned16(out) || lse == nullptr || !aligned4(lse)) return LS_ERR_INVALID_ARG;
   rc = run_partials(q, k_cache, v_cache, k_tree, v_tree, tree_parent, cu_seqlens, dims, paged, workspace,
-                    workspace_bytes, stream, true, tree);
+                    workspace_bytes, stream, true, tree, &p);
   if (rc != LS_OK) return rc;
-  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, true, tree);
+  return run_combine(cu_seqlens, out, lse, dims, workspace, workspace_bytes, stream, true, tree, &p);
 }
 
 int ls_verify_attn_check(const ls_verify_dims* dims, const void* workspace, void* stream) {

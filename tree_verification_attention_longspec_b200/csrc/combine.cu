@@ -19,6 +19,25 @@
 namespace ls {
 namespace {
 
+// The merge's exponentials, reciprocal and logarithm by the special-function unit's
+// approximate instructions (relative error about 2^-22, far below the bf16 result's 2^-9):
+// the accurate library versions lengthened each row's dependent chain measurably.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_fast(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_fast(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 constexpr int kPrefetch = 20;  // partials in flight per warp (the headline has 18 per row)
 
 template <int D, bool WIDE>
@@ -123,8 +142,8 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
         const float Mn = fmaxf(M, mx);
-        const float corr = M == Mn ? 1.f : exp2f(M - Mn);       // M = -inf before any weight: 0
-        const float wl = lx == -INFINITY ? 0.f : exp2f(lx - Mn);  // this lane's chunk weight
+        const float corr = M == Mn ? 1.f : ex2_fast(M - Mn);       // M = -inf before any weight: 0
+        const float wl = lx == -INFINITY ? 0.f : ex2_fast(lx - Mn);  // this lane's chunk weight
         Lsum = Lsum * corr + warp_sum(wl);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] *= corr;
@@ -162,7 +181,7 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
       for (int e = 0; e < E; ++e) acc[e] = 0.f;
       for (int w = 0; w < kMergeRows; ++w) {
         if (!(w_l[w] > 0.f)) continue;  // a warp without partials
-        const float f = exp2f(w_m[w] - Mt);
+        const float f = ex2_fast(w_m[w] - Mt);
         Lsum = fmaf(w_l[w], f, Lsum);
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = fmaf(w_acc[w][lane * E + e], f, acc[e]);
@@ -171,14 +190,14 @@ __global__ void __maxnreg__(112) combine_kernel(const __grid_constant__ CombineA
     }
   }
   if (writes && (!wide || warp == 0)) {
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    const float inv = Lsum > 0.f ? rcp_fast(Lsum) : 0.f;
     uint16_t* dst = a.out + out_row * D + lane * E;
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
       const uint32_t lo = f32_to_bf16(acc[e] * inv), hi = f32_to_bf16(acc[e + 1] * inv);
       *reinterpret_cast<uint32_t*>(dst + e) = lo | (hi << 16);
     }
-    if (lane == 0) a.lse[out_row] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+    if (lane == 0) a.lse[out_row] = Lsum > 0.f ? (M + lg2_fast(Lsum)) * kLn2 : -INFINITY;
   }
 #pragma unroll
   for (int o2 = 16; o2 > 0; o2 >>= 1) err |= __shfl_xor_sync(0xffffffffu, err, o2);

@@ -7,10 +7,11 @@
 // of them, row (i - u*tpu)*g + j of the unit) and one TMA box brings them in.
 // The keys of sequence b form ceil(L_b / 128) prefix blocks ("Cached-Teil", no mask)
 // followed by one block of its T <= 128 tree keys ("Speculative-Teil", tree mask).
-// Every chunk of a sequence covers C consecutive blocks of that list, so the chunk
-// that holds the tree block also attends the last prefix keys, and a sequence without
-// prefix still has one chunk. The chunk grid follows from the prefix lengths and C
-// alone, and the device recomputes it from cu_seqlens without any table in memory.
+// A sequence's list is cut into n = ceil(blocks / C) chunks of consecutive blocks, as
+// even as possible, so the chunk that holds the tree block also attends the last prefix
+// keys, and a sequence without prefix still has one chunk. The chunk grid follows from
+// the prefix lengths and C alone, and the device recomputes it from cu_seqlens without
+// any table in memory.
 // Trees may differ in size per sequence (cu_tree): the grid is then planned for T, the
 // largest tree allowed, and units past a sequence's own tree have no rows.
 #pragma once
@@ -177,7 +178,10 @@ LS_HD ChunkCoord locate_chunk(const Plan& p, const int32_t* cu, int32_t cid) {
       c.key_skip = window_start(p, L);
       c.seq_offset = cu[b] + c.key_skip;
       const int32_t Lc = attended_len(p, L);
-      const int32_t v0 = c.split * p.C, v1 = v0 + p.C;  // blocks [v0, v1) of the key list
+      // The key list's blocks are cut into n runs of consecutive blocks as even as
+      // possible (their lengths differ by at most one, none longer than C): blocks [v0, v1).
+      const int32_t nbl = prefix_blocks(Lc) + p.with_tree;
+      const int32_t v0 = (int32_t)((int64_t)c.split * nbl / n), v1 = (int32_t)((int64_t)(c.split + 1) * nbl / n);
       const int32_t kb = v0 * kBlockN, ke = v1 * kBlockN;
       c.key_begin = kb < Lc ? kb : Lc;
       c.key_end = ke < Lc ? ke : Lc;
