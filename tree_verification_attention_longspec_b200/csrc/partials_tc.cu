@@ -659,16 +659,17 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
         const int lim = j == nb - 1 ? tail_end : kBlockN;  // columns from here on are masked
         const bool tree_blk = j == nb;                      // keys = the sequence's tree nodes
         if (tree_blk && mask_tree_scores(bars->parent, tS, has_row ? node : -1)) bars->tree_err = 1u;
-        // All 128 scores for the row maximum; the scores of keys 0..63 stay in registers
-        // for P's first half, those of keys 64..127 are read again for the second half.
+        // All 128 scores for the row maximum, kept in registers for both halves of P (P
+        // goes to columns 0..63, whose scores are in registers by then; d = 64 reads keys
+        // 64..127 again below).
         float lo[kHalf];
+        float hi[kHalf];
         float mx;
         {
           uint32_t r[4][32];
 #pragma unroll
           for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, r[q]);
           tmem_wait_ld();
-          float hi[kHalf];
 #pragma unroll
           for (int e = 0; e < kHalf; ++e) {
             lo[e] = __uint_as_float(r[e >> 5][e & 31]);
@@ -723,15 +724,16 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
             m = m_new;
           }
           tmem_st32(tS, pk);  // P over keys 0..63 -> columns 0..31
-        }
-        float hi[kHalf];
-        {
-          uint32_t r[2][32];
-          tmem_ld32(tS + 64, r[0]);  // P occupies columns 0..63 only: keys 64..127 are intact
-          tmem_ld32(tS + 96, r[1]);
           tmem_wait_st();
           tc_fence_before_sync();
           mbar_arrive(&bars->p_full[t][0]);
+        }
+        if constexpr (D != 128) {
+          // d = 64 would spill with both halves live: its keys 64..127 are read again (P
+          // took columns 0..31 only, so their scores are intact)
+          uint32_t r[2][32];
+          tmem_ld32(tS + 64, r[0]);
+          tmem_ld32(tS + 96, r[1]);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < kHalf; ++e) hi[e] = __uint_as_float(r[e >> 5][e & 31]);
