@@ -211,7 +211,11 @@ __device__ __forceinline__ bool mask_tree_scores(const int16_t* parent, uint32_t
   return bad;
 }
 
-template <int D, int EMU>
+// GENERAL = false: the instance for a packed cache, the whole prefix and inputs as given;
+// the paged, sliding-window and rotated-input paths are compiled out of it, which keeps
+// the code the block loop fetches smaller (2% on the Qwen-7B layer). GENERAL = true: every
+// path, chosen at run time.
+template <int D, int EMU, bool GENERAL>
 __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_constant__ TcParams P) {
   using C = Cfg<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   // sequence end (its leading tail_shift columns are earlier keys, masked); in a paged
   // cache it is loaded from its aligned start, page by page, and its columns from
   // tail_end on lie past the sequence end (masked).
-  const bool paged = a.page_table != nullptr;
+  const bool paged = GENERAL && a.page_table != nullptr;
   const int tail_shift = paged ? 0 : nb * kBlockN - n_keys;
   const int tail_end = paged ? n_keys - (nb - 1) * kBlockN : kBlockN;
   const bool has_tree = c.has_tree;
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   const int seq_len = cu[c.b + 1] - cu[c.b];
   // sliding window: a row at depth d sees the attended keys from window_cut(d) on, which
   // is below 2 * 128, so only the chunks that start there cut rows individually
-  const bool win_rows = p.window > 0 && nb > 0 && c.key_begin < 2 * kBlockN;
+  const bool win_rows = GENERAL && p.window > 0 && nb > 0 && c.key_begin < 2 * kBlockN;
   int tree_base, tree_n;  // the sequence's tree nodes (none if cu_tree is bad: the combine reports it)
   tree_range(p, a.cu_tree, c.b, &tree_base, &tree_n);
   const int tok0 = c.rgi * p.tpu;                       // first tree node of the unit
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   };
   // When the tree kernel writes q and k_tree (rotated), this grid may start before
   // that grid ends: the prefix loads go ahead, Q and the tree block wait for it.
-  bool prior_done = !a.after_prep;
+  bool prior_done = !GENERAL || !a.after_prep;
   auto wait_prior = [&]() {
     if (!prior_done) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -865,7 +869,7 @@ bool make_o_map(CUtensorMap* map, float* base, int D, int64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int EMU>
+template <int D, int EMU, bool GENERAL>
 cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream) {
   TcParams P;
   P.a = a;
@@ -884,12 +888,12 @@ cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(partials_tc_kernel<D, EMU>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(partials_tc_kernel<D, EMU, GENERAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   if (!a.after_prep) {
-    partials_tc_kernel<D, EMU><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
+    partials_tc_kernel<D, EMU, GENERAL><<<a.p.n_chunks, kThreads, smem, stream>>>(P);
     return cudaGetLastError();
   }
   // a programmatic dependent of the tree kernel (see the producer's wait_prior)
@@ -903,7 +907,7 @@ cudaError_t launch_d(const PartialsArgs& a, int64_t kv_rows, cudaStream_t stream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, partials_tc_kernel<D, EMU>, P);
+  return cudaLaunchKernelEx(&cfg, partials_tc_kernel<D, EMU, GENERAL>, P);
 }
 
 }  // namespace
@@ -914,8 +918,9 @@ cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t
   // softmax's exponentials move off the special-function unit (MUFU), which is as busy
   // as the tensor pipe at d = 128 and busier at d = 64. More than a quarter makes the
   // FMA pipe the slower one.
-  if (a.p.d == 64) return launch_d<64, 1>(a, kv_rows, stream);
-  return launch_d<128, 1>(a, kv_rows, stream);
+  const bool general = a.page_table != nullptr || a.p.window > 0 || a.after_prep;
+  if (a.p.d == 64) return general ? launch_d<64, 1, true>(a, kv_rows, stream) : launch_d<64, 1, false>(a, kv_rows, stream);
+  return general ? launch_d<128, 1, true>(a, kv_rows, stream) : launch_d<128, 1, false>(a, kv_rows, stream);
 }
 
 }  // namespace ls
