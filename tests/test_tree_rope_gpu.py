@@ -212,3 +212,25 @@ def test_sliding_window_d64_device_lengths():
     assert st == binding.LS_OK
     ro, rl = _oracle(inp, window=100)
     _assert_close(o, l_, ro, rl)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,T,lengths", [(2, 28, 4, 128, 64, [3000, 9000]),
+                                                   (3, 8, 2, 64, 16, [130, 0, 5000])])
+def test_plain_and_general_instances_agree_bitwise(B, Hq, Hkv, d, T, lengths):
+    """The partials kernel is compiled twice: a plain instance (packed cache, whole prefix,
+    inputs as given) and a general one (paged caches, windows, rotation). A window longer
+    than every key list and a paged cache of 128-key pages ask for the general instance
+    without changing what is computed: both must give the plain call's bits."""
+    w = Workload("instances", B, Hq, Hkv, d, T, 0, "window8", input_scale=1.0, lengths=lengths)
+    inp = make_inputs(w, seed=30 + d)
+    o_plain, l_plain, st, _ = _run_ex(inp)
+    assert st == binding.LS_OK
+    o_win, l_win, st, _ = _run_ex(inp, window=max(lengths) + T + 1)
+    assert st == binding.LS_OK
+    o_pg, l_pg, st, _ = _run_ex(inp, page_size=128)
+    assert st == binding.LS_OK
+    for o, l_ in ((o_win, l_win), (o_pg, l_pg)):
+        np.testing.assert_array_equal(o, o_plain)
+        np.testing.assert_array_equal(l_, l_plain)
+    ro, rl = _oracle(inp)
+    _assert_close(o_plain, l_plain, ro, rl)
