@@ -215,22 +215,29 @@ def test_sliding_window_d64_device_lengths():
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,d,T,lengths", [(2, 28, 4, 128, 64, [3000, 9000]),
-                                                   (3, 8, 2, 64, 16, [130, 0, 5000])])
+                                                   (3, 8, 2, 64, 16, [130, 0, 5000]),
+                                                   (2, 28, 4, 128, 64, [3072, 8960])])
 def test_plain_and_general_instances_agree_bitwise(B, Hq, Hkv, d, T, lengths):
     """The partials kernel is compiled twice: a plain instance (packed cache, whole prefix,
     inputs as given) and a general one (paged caches, windows, rotation). A window longer
-    than every key list and a paged cache of 128-key pages ask for the general instance
-    without changing what is computed: both must give the plain call's bits."""
+    than every key list asks for the general instance without changing what is computed,
+    or where the keys sit in a block: it must give the plain call's bits. So must a paged
+    cache of 128-key pages when every length is a multiple of 128 (otherwise its last
+    block holds the keys at other columns, masked at the end instead of the start, and
+    the sums round differently)."""
     w = Workload("instances", B, Hq, Hkv, d, T, 0, "window8", input_scale=1.0, lengths=lengths)
     inp = make_inputs(w, seed=30 + d)
     o_plain, l_plain, st, _ = _run_ex(inp)
     assert st == binding.LS_OK
     o_win, l_win, st, _ = _run_ex(inp, window=max(lengths) + T + 1)
     assert st == binding.LS_OK
+    np.testing.assert_array_equal(o_win, o_plain)
+    np.testing.assert_array_equal(l_win, l_plain)
     o_pg, l_pg, st, _ = _run_ex(inp, page_size=128)
     assert st == binding.LS_OK
-    for o, l_ in ((o_win, l_win), (o_pg, l_pg)):
-        np.testing.assert_array_equal(o, o_plain)
-        np.testing.assert_array_equal(l_, l_plain)
+    if all(L % 128 == 0 for L in lengths):
+        np.testing.assert_array_equal(o_pg, o_plain)
+        np.testing.assert_array_equal(l_pg, l_plain)
     ro, rl = _oracle(inp)
     _assert_close(o_plain, l_plain, ro, rl)
+    _assert_close(o_pg, l_pg, ro, rl)
