@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 
 import oracle
-from tests.gpu_harness import LSE_ATOL, OUT_ATOL, make_op, out_tolerance, run_gpu, to_device
+from tests.gpu_harness import LSE_ATOL, OUT_ATOL, make_op, out_tolerance, run_gpu, spread_tolerance, to_device, value_spread
 from tree_verification_attention_longspec_b200.inputs import Workload, bf16_bits_to_f32, make_inputs
 from tree_verification_attention_longspec_b200.workloads import WORKLOADS
 
@@ -170,5 +170,62 @@ def test_workspace_contents_do_not_matter():
     op = make_op(inp, host_lengths=False)
     op.workspace.fill_(0xFF)
     out, lse, st = run_gpu(inp, dev=dev, op=op)
+    assert st == 0
+    _compare(inp, out, lse)
+
+
+@pytest.mark.parametrize("scale", [2.0, 3.0])
+def test_peaked_softmax_all_rows(scale):
+    """Inputs drawn N(0, scale^2), beyond the workloads' N(0, 1): the scores' spread grows
+    as scale^2 (std 4 and 9), so rows are dominated by a few keys, the running max is
+    raised well past the lazy threshold as the blocks go by, and the weights' bf16
+    rounding does not average out. The values spread as widely (std scale), and a fixed
+    1e-2 no longer holds: the bound is the one the weights' rounding gives, half an ulp
+    plus 2^-7 of the values' weighted spread (gpu_harness.spread_tolerance)."""
+    inp = _small(2, 28, 4, 128, 64, [3000, 9000], "window8", seed=int(scale * 10), scale=scale)
+    out, lse, st = run_gpu(inp)
+    assert st == 0
+    ro, rl = oracle.verify_attn_oracle_inputs(inp)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    mean, spread = value_spread(inp)
+    assert np.abs(mean - ro).max() < 1e-9  # the helper's weights are the oracle's
+    tol = spread_tolerance(ro, spread)
+    err = np.abs(out - ro)
+    assert np.all(err <= tol), f"out error {err.flat[(err - tol).argmax()]} over {tol.flat[(err - tol).argmax()]}"
+    assert np.abs(lse - rl).max() <= LSE_ATOL
+
+
+def test_keys_growing_along_the_sequence_all_rows():
+    """Key vectors scaled by a ramp from 0.25 to 3 along each sequence: every block tends
+    to raise the running max of its rows, so the O rescale runs block after block."""
+    from tree_verification_attention_longspec_b200.inputs import bf16_bits_from_f32, bf16_bits_to_f32
+    inp = _small(2, 16, 2, 128, 32, [5000, 2500], "bfs", seed=44)
+    k = bf16_bits_to_f32(inp.k_cache)
+    for b in range(2):
+        s0, s1 = int(inp.cu_seqlens[b]), int(inp.cu_seqlens[b + 1])
+        ramp = np.linspace(0.25, 3.0, s1 - s0, dtype=np.float32)[:, None, None]
+        k[s0:s1] *= ramp
+    inp.k_cache = bf16_bits_from_f32(k)
+    out, lse, st = run_gpu(inp)
+    assert st == 0
+    _compare(inp, out, lse)
+
+
+@pytest.mark.parametrize("host_lengths", [True, False])
+def test_group_256_one_node_per_unit(host_lengths):
+    # g = 256, the largest group: a unit holds one tree node's 256 heads
+    inp = _small(2, 256, 1, 64, 3, [700, 129], "chain", seed=45)
+    out, lse, st = run_gpu(inp, host_lengths=host_lengths)
+    assert st == 0
+    _compare(inp, out, lse)
+
+
+@pytest.mark.parametrize("B", [32, 33])
+def test_batch_at_the_plan_s_host_length_limit(B):
+    # the plan carries host lengths for B <= 32 and reads the device array beyond
+    rng = np.random.default_rng(B)
+    lengths = [int(x) for x in rng.integers(0, 1500, size=B)]
+    inp = _small(B, 8, 2, 128, 4, lengths, "uniform", seed=B)
+    out, lse, st = run_gpu(inp)
     assert st == 0
     _compare(inp, out, lse)
