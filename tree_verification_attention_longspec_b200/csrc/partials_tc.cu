@@ -211,10 +211,10 @@ __device__ __forceinline__ bool mask_tree_scores(const int16_t* parent, uint32_t
   return bad;
 }
 
-// GENERAL = false: the instance for a packed cache, the whole prefix and inputs as given;
-// the paged, sliding-window and rotated-input paths are compiled out of it, which keeps
-// the code the block loop fetches smaller (2% on the Qwen-7B layer). GENERAL = true: every
-// path, chosen at run time.
+// GENERAL = false: the instance for a packed cache and the whole prefix; the paged and
+// sliding-window paths are compiled out of it, which keeps the code the block loop
+// fetches smaller (2% on the Qwen-7B layer). GENERAL = true: every path, chosen at run
+// time. Both wait for the tree kernel when it rotates q and k_tree first.
 template <int D, int EMU, bool GENERAL>
 __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_constant__ TcParams P) {
   using C = Cfg<D>;
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) partials_tc_kernel(const __grid_c
   };
   // When the tree kernel writes q and k_tree (rotated), this grid may start before
   // that grid ends: the prefix loads go ahead, Q and the tree block wait for it.
-  bool prior_done = !GENERAL || !a.after_prep;
+  bool prior_done = !a.after_prep;
   auto wait_prior = [&]() {
     if (!prior_done) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -918,7 +918,7 @@ cudaError_t launch_partials(const PartialsArgs& a, int64_t kv_rows, cudaStream_t
   // softmax's exponentials move off the special-function unit (MUFU), which is as busy
   // as the tensor pipe at d = 128 and busier at d = 64. More than a quarter makes the
   // FMA pipe the slower one.
-  const bool general = a.page_table != nullptr || a.p.window > 0 || a.after_prep;
+  const bool general = a.page_table != nullptr || a.p.window > 0;
   if (a.p.d == 64) return general ? launch_d<64, 1, true>(a, kv_rows, stream) : launch_d<64, 1, false>(a, kv_rows, stream);
   return general ? launch_d<128, 1, true>(a, kv_rows, stream) : launch_d<128, 1, false>(a, kv_rows, stream);
 }
